@@ -1,0 +1,264 @@
+/*
+ * attn_oracle.c -- fp64 CPU oracle for exact scaled dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or constant with the CUDA kernels it checks.
+ *
+ * What it computes (exact attention, the computation FlashAttention-4 speeds
+ * up without changing its result -- "FlashAttention-4 Overcomes Memory
+ * Bottlenecks", body; "The Technical Edge", adaptive rescaling that keeps
+ * numerical stability), for one (batch, head) slice with row-major n x d
+ * operands q, k, v (and dO for the backward):
+ *
+ *   S_ij   = scale * sum_c q_ic k_jc            j visible to i
+ *   visible: every j, or j <= i when causal (queries and keys aligned at the
+ *            first position; a masked key contributes nothing)
+ *   m_i    = max_j S_ij
+ *   LSE_i  = m_i + ln sum_j exp(S_ij - m_i)    (natural logarithm)
+ *   P_ij   = exp(S_ij - LSE_i)
+ *   O_i    = sum_j P_ij v_j
+ *
+ * Backward (chain rule through the softmax, P recomputed from LSE):
+ *   dP_ij  = dO_i . v_j
+ *   D_i    = sum_j P_ij dP_ij
+ *   dS_ij  = P_ij (dP_ij - D_i)
+ *   dQ_i   = scale * sum_j dS_ij k_j
+ *   dK_j   = scale * sum_i dS_ij q_i
+ *   dV_j   = sum_i P_ij dO_i
+ *
+ * Everything is plain fp64 loops in the order written above.  The only
+ * structure added is threading: rows (forward, dQ) and key columns (dK, dV)
+ * are split across POSIX threads; each output element is computed by exactly
+ * one thread, so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    const double *q, *k, *v, *dout;
+    int64_t n, d;
+    double scale;
+    int causal;
+    const int64_t *rows;   /* which rows (forward / dQ) or key columns (dK, dV) */
+    int64_t count;
+    double *out_a;         /* O rows, or dQ rows, or dK rows */
+    double *out_b;         /* LSE,    or unused,  or dV rows */
+    double *lse_all;       /* backward: LSE_i for every row i */
+    double *dsum_all;      /* backward: D_i for every row i */
+    int tid, nthreads;
+    int status;
+} job_t;
+
+static double dot(const double *a, const double *b, int64_t d)
+{
+    double s = 0.0;
+    for (int64_t c = 0; c < d; ++c) s += a[c] * b[c];
+    return s;
+}
+
+/* number of keys visible to query row i */
+static int64_t visible(int64_t i, int64_t n, int causal) { return causal ? i + 1 : n; }
+
+/* S_i. (visible part), returns LSE_i; s has room for n values */
+static double score_row(const job_t *J, int64_t i, double *s)
+{
+    const double *qi = J->q + i * J->d;
+    int64_t nv = visible(i, J->n, J->causal);
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nv; ++j) {
+        s[j] = J->scale * dot(qi, J->k + j * J->d, J->d);
+        if (s[j] > m) m = s[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < nv; ++j) l += exp(s[j] - m);
+    return m + log(l);
+}
+
+/* ---------------------------------------------------------------- forward */
+static void *fwd_worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(J->n > 0 ? J->n : 1));
+    if (!s) { J->status = 1; return NULL; }
+    for (int64_t r = J->tid; r < J->count; r += J->nthreads) {
+        int64_t i = J->rows ? J->rows[r] : r;
+        double lse = score_row(J, i, s);
+        double *o = J->out_a + r * J->d;
+        for (int64_t c = 0; c < J->d; ++c) o[c] = 0.0;
+        int64_t nv = visible(i, J->n, J->causal);
+        for (int64_t j = 0; j < nv; ++j) {
+            double p = exp(s[j] - lse);
+            const double *vj = J->v + j * J->d;
+            for (int64_t c = 0; c < J->d; ++c) o[c] += p * vj[c];
+        }
+        J->out_b[r] = lse;
+    }
+    free(s);
+    return NULL;
+}
+
+/* ------------------------------------------------- backward, pass 1 (rows) */
+/* LSE_i and D_i for every row; dQ_i for the requested rows (out_a, indexed by
+ * the position of i in rows[]; rowpos maps i -> position or -1). */
+typedef struct { job_t base; const int64_t *rowpos; } job1_t;
+
+static void *bwd_rows_worker(void *arg)
+{
+    job1_t *J1 = (job1_t *)arg;
+    job_t *J = &J1->base;
+    double *s = (double *)malloc(sizeof(double) * (size_t)J->n);
+    double *ds = (double *)malloc(sizeof(double) * (size_t)J->n);
+    if (!s || !ds) { free(s); free(ds); J->status = 1; return NULL; }
+    for (int64_t i = J->tid; i < J->n; i += J->nthreads) {
+        int64_t nv = visible(i, J->n, J->causal);
+        double lse = score_row(J, i, s);
+        const double *doi = J->dout + i * J->d;
+        double D = 0.0;
+        for (int64_t j = 0; j < nv; ++j) {
+            double p = exp(s[j] - lse);
+            double dp = dot(doi, J->v + j * J->d, J->d);
+            s[j] = p;          /* P_ij */
+            ds[j] = dp;        /* dP_ij */
+            D += p * dp;
+        }
+        J->lse_all[i] = lse;
+        J->dsum_all[i] = D;
+        int64_t pos = J1->rowpos ? J1->rowpos[i] : -1;
+        if (pos >= 0) {
+            double *dq = J->out_a + pos * J->d;
+            for (int64_t c = 0; c < J->d; ++c) dq[c] = 0.0;
+            for (int64_t j = 0; j < nv; ++j) {
+                double dsij = s[j] * (ds[j] - D);
+                const double *kj = J->k + j * J->d;
+                for (int64_t c = 0; c < J->d; ++c) dq[c] += dsij * kj[c];
+            }
+            for (int64_t c = 0; c < J->d; ++c) dq[c] *= J->scale;
+        }
+    }
+    free(s); free(ds);
+    return NULL;
+}
+
+/* ---------------------------------------------- backward, pass 2 (columns) */
+static void *bwd_cols_worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    for (int64_t r = J->tid; r < J->count; r += J->nthreads) {
+        int64_t j = J->rows ? J->rows[r] : r;
+        const double *kj = J->k + j * J->d;
+        const double *vj = J->v + j * J->d;
+        double *dk = J->out_a + r * J->d;
+        double *dv = J->out_b + r * J->d;
+        for (int64_t c = 0; c < J->d; ++c) { dk[c] = 0.0; dv[c] = 0.0; }
+        int64_t i0 = J->causal ? j : 0;          /* rows that see key j */
+        for (int64_t i = i0; i < J->n; ++i) {
+            const double *qi = J->q + i * J->d;
+            const double *doi = J->dout + i * J->d;
+            double p = exp(J->scale * dot(qi, kj, J->d) - J->lse_all[i]);
+            double dp = dot(doi, vj, J->d);
+            double dsij = p * (dp - J->dsum_all[i]);
+            for (int64_t c = 0; c < J->d; ++c) {
+                dk[c] += dsij * qi[c];
+                dv[c] += p * doi[c];
+            }
+        }
+        for (int64_t c = 0; c < J->d; ++c) dk[c] *= J->scale;
+    }
+    return NULL;
+}
+
+static int run_threads(void *(*fn)(void *), void *jobs, size_t job_size, int nthreads)
+{
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) return 1;
+    int started = 0, st = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&th[t], NULL, fn, (char *)jobs + job_size * (size_t)t) != 0) { st = 1; break; }
+        started++;
+    }
+    for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+    free(th);
+    for (int t = 0; t < started; ++t) st |= ((job_t *)((char *)jobs + job_size * (size_t)t))->status;
+    return st;
+}
+
+static int check_args(const double *q, const double *k, const double *v, int64_t n, int64_t d, int nthreads)
+{
+    if (!q || !k || !v) return 1;
+    if (n < 1 || d < 1 || nthreads < 1) return 1;
+    return 0;
+}
+
+/*
+ * Forward for one head.  rows == NULL computes every row (count must be n);
+ * otherwise row r of o (count x d) and lse (count) belongs to query rows[r].
+ * Returns 0 on success.
+ */
+int oracle_attn_fwd(const double *q, const double *k, const double *v, int64_t n, int64_t d,
+                    double scale, int causal, const int64_t *rows, int64_t count,
+                    double *o, double *lse, int nthreads)
+{
+    if (check_args(q, k, v, n, d, nthreads) || !o || !lse || count < 0) return 1;
+    if (!rows && count != n) return 1;
+    for (int64_t r = 0; rows && r < count; ++r) if (rows[r] < 0 || rows[r] >= n) return 1;
+    job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+    if (!jobs) return 1;
+    for (int t = 0; t < nthreads; ++t) {
+        job_t J = {q, k, v, NULL, n, d, scale, causal, rows, count, o, lse, NULL, NULL, t, nthreads, 0};
+        jobs[t] = J;
+    }
+    int st = run_threads(fwd_worker, jobs, sizeof(job_t), nthreads);
+    free(jobs);
+    return st;
+}
+
+/*
+ * Backward for one head.  Computes LSE_i and D_i for all rows (written to
+ * lse_all / dsum_all, n values each), dQ for the nq rows listed in qrows
+ * (NULL: all rows, nq == n) and dK, dV for the nk key rows listed in krows
+ * (NULL: all, nk == n).  Returns 0 on success.
+ */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    int64_t n, int64_t d, double scale, int causal,
+                    const int64_t *qrows, int64_t nq, const int64_t *krows, int64_t nk,
+                    double *dq, double *dk, double *dv, double *lse_all, double *dsum_all,
+                    int nthreads)
+{
+    if (check_args(q, k, v, n, d, nthreads) || !dout || !lse_all || !dsum_all) return 1;
+    if ((nq > 0 && !dq) || (nk > 0 && (!dk || !dv)) || nq < 0 || nk < 0) return 1;
+    if ((!qrows && nq != n && nq != 0) || (!krows && nk != n && nk != 0)) return 1;
+    int64_t *rowpos = (int64_t *)malloc(sizeof(int64_t) * (size_t)n);
+    if (!rowpos) return 1;
+    for (int64_t i = 0; i < n; ++i) rowpos[i] = -1;
+    for (int64_t r = 0; r < nq; ++r) {
+        int64_t i = qrows ? qrows[r] : r;
+        if (i < 0 || i >= n) { free(rowpos); return 1; }
+        rowpos[i] = r;
+    }
+    for (int64_t r = 0; krows && r < nk; ++r) if (krows[r] < 0 || krows[r] >= n) { free(rowpos); return 1; }
+
+    job1_t *j1 = (job1_t *)calloc((size_t)nthreads, sizeof(job1_t));
+    job_t *j2 = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+    int st = 1;
+    if (j1 && j2) {
+        for (int t = 0; t < nthreads; ++t) {
+            job_t J = {q, k, v, dout, n, d, scale, causal, NULL, n, dq, NULL, lse_all, dsum_all, t, nthreads, 0};
+            j1[t].base = J;
+            j1[t].rowpos = rowpos;
+        }
+        st = run_threads(bwd_rows_worker, j1, sizeof(job1_t), nthreads);
+        if (st == 0 && nk > 0) {
+            for (int t = 0; t < nthreads; ++t) {
+                job_t J = {q, k, v, dout, n, d, scale, causal, krows, nk, dk, dv, lse_all, dsum_all, t, nthreads, 0};
+                j2[t] = J;
+            }
+            st = run_threads(bwd_cols_worker, j2, sizeof(job_t), nthreads);
+        }
+    }
+    free(j1); free(j2); free(rowpos);
+    return st;
+}
