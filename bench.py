@@ -1,0 +1,355 @@
+"""Benchmark: exact attention forward + backward on B200 (libfa, sm_100a).
+
+One step = the whole hot path on one batch: fa_fwd (O, LSE) then fa_bwd
+(dQ, dK, dV) on the long-context causal workload B=1, H=16, N=32768, d=128,
+bf16, scale 1/sqrt(d), seeded N(0, 1) inputs.  FLOPs follow the usual
+convention: forward 4*B*H*N^2*d, backward 2.5x that, both halved for causal.
+
+Prints one JSON line (rank 0).  `value` is device-timed throughput (CUDA
+events around exactly --steps steps, inputs resident in HBM, max over ranks);
+`e2e` is the same metric through the C ABI with host buffers (pinned
+host->device copy of Q, K, V, dO and device->host copy of O, LSE, dQ, dK, dV
+inside the timed region).  Multi-GPU (torchrun): every rank runs its own
+batch of heads (no collective on the data path), weak scaling.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="long-context fwd+bwd causal", B=1, H=16, N=32768, d=128, causal=True, seed_workload=4)
+METRIC = "attention fwd/bwd TFLOPS (bf16, 1xB200) and % of dense BF16 tensor peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
+    return f, 2.5 * f
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return dict(burst=float(p["bf16_tflops"]), sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(burst=1590.0, sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def config_dict(n_gpus):
+    w = WORKLOAD
+    return {"workload": f"{w['name']}: B={w['B']} H={w['H']} N={w['N']} d={w['d']}",
+            "B": w["B"], "H": w["H"], "seq_len": w["N"], "head_dim": w["d"], "causal": w["causal"],
+            "global_batch_heads": w["B"] * w["H"] * n_gpus, "parallelism": f"heads sharded x{n_gpus} (no collective)",
+            "l2": "inputs larger than L2 (Q, K, V, dO 134 MB each vs 126 MB L2); no explicit flush"}
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = sorted(sm)[len(sm) // 4:] or sm  # drop the idle head of the record
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_159_b200 import api, build, inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    build.build()
+    w = WORKLOAD
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    scale = 1.0 / math.sqrt(d)
+    # each rank draws its own heads (weak scaling): shift the seed by rank
+    bits = I.attention_inputs(w["seed_workload"] + 100 * rank, B, H, N, d, with_do=True)
+    host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in bits.items()}
+    dev = {k: v.cuda() for k, v in host.items()}
+    o = torch.empty_like(dev["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = (torch.empty_like(dev["q"]) for _ in range(3))
+    ws = torch.empty(api.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(prof=None):
+        if prof is not None:
+            api.fa_profile_next(0, prof[0], prof[1])
+            api.fa_profile_next(1, prof[2], prof[3])
+        api.fa_fwd(dev["q"], dev["k"], dev["v"], scale, causal, out=o, lse=lse)
+        api.fa_bwd(dev["q"], dev["k"], dev["v"], o, dev["do"], lse, scale, causal, dq=dq, dk=dk, dv=dv,
+                   workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    rc, detail = api.fa_last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x}) after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e4 in ev:  # torch creates the CUDA event handle at its first record
+        for e in e4:
+            e.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(ev[i])
+        t1.record(stream)
+        barrier()
+    rc, detail = api.fa_last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x}) in the timed region")
+    ms = t0.elapsed_time(t1)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in ev]
+
+    # end to end through host buffers
+    h_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in
+             (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(host[k].numel() * host[k].element_size() for k in ("q", "k", "v", "do"))
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    def e2e_step():
+        for k in ("q", "k", "v", "do"):
+            dev[k].copy_(host[k], non_blocking=True)
+        step()
+        h_out["o"].copy_(o, non_blocking=True)
+        h_out["lse"].copy_(lse, non_blocking=True)
+        h_out["dq"].copy_(dq, non_blocking=True)
+        h_out["dk"].copy_(dk, non_blocking=True)
+        h_out["dv"].copy_(dv, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    vals = torch.tensor([ms, e2e_ms, max(fwd_ms), max(bwd_ms)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, e2e_ms = float(vals[0]), float(vals[1])
+    f_fwd, f_bwd = flops(B, H, N, d, causal)
+    step_flops = (f_fwd + f_bwd) * world
+    ms_step = ms / args.steps
+    value = step_flops / (ms_step * 1e-3) / 1e12
+    pk = peaks()
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+    fwd_tf = f_fwd / (fwd_avg * 1e-3) / 1e12
+    bwd_tf = f_bwd / (bwd_avg * 1e-3) / 1e12
+    dominant = "bwd" if bwd_avg >= fwd_avg else "fwd"
+    ach = bwd_tf if dominant == "bwd" else fwd_tf
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": config_dict(world),
+        "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+        "fwd_ms": round(fwd_avg, 4), "bwd_main_ms": round(bwd_avg, 4),
+        "pct_dense_bf16_peak": {"step": round(100 * value / world / DATASHEET_BF16_TFLOPS, 2),
+                                "fwd": round(100 * fwd_tf / DATASHEET_BF16_TFLOPS, 2),
+                                "bwd": round(100 * bwd_tf / DATASHEET_BF16_TFLOPS, 2),
+                                "denominator": "2250 TFLOPS datasheet dense bf16",
+                                "fwd_of_measured_burst": round(100 * fwd_tf / pk["burst"], 2),
+                                "bwd_of_measured_burst": round(100 * bwd_tf / pk["burst"], 2)},
+        "roofline": {"bound": "tensor", "kernel": f"{dominant} attention kernel", "achieved": round(ach, 2),
+                     "peak": pk["sustained"], "unit": "TFLOP/s", "frac": round(ach / pk["sustained"], 4),
+                     "peak_kind": f"{pk['source']} sustained bf16 (kernel timed inside a multi-second loop)",
+                     "traffic": None},
+        "e2e": {"value": round(step_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+                "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ---------------------------------------------------------------- CPU oracle
+def _oracle_sample(budget_s):
+    """Oracle forward on query rows of head (0, 0) of the workload, every `stride`-th row,
+    stride chosen so the sample is ~budget_s of work on this host."""
+    import numpy as np
+
+    from exact_attention_159_b200 import inputs as I
+    from oracle import oracle as OR
+
+    w = WORKLOAD
+    N, d = w["N"], w["d"]
+    seed = w["seed_workload"]
+    # head (0, 0) is the first N*d draws of each tensor's stream
+    q, k, v = (I.bf16_bits_to_f64(I.normal_bf16(I.seed_for(seed, t), (N, d))) for t in ("q", "k", "v"))
+    threads = OR.default_threads()
+    # calibrate on a small row set
+    probe = np.arange(0, N, 512)
+    t = time.perf_counter()
+    OR.fwd(q, k, v, 1.0 / math.sqrt(d), w["causal"], rows=probe, nthreads=threads)
+    dt = max(time.perf_counter() - t, 1e-3)
+    stride = max(1, int(512 * dt / budget_s))
+    rows = np.arange(stride // 2, N, stride)
+    return q, k, v, rows, stride, threads
+
+
+def cpu_baseline(budget_s=15.0):
+    import numpy as np
+
+    from oracle import oracle as OR
+
+    q, k, v, rows, stride, threads = _oracle_sample(budget_s)
+    w = WORKLOAD
+    t = time.perf_counter()
+    OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
+    dt = time.perf_counter() - t
+    vis = (rows + 1) if w["causal"] else np.full(rows.shape, w["N"])
+    fl = float(4.0 * w["d"] * vis.sum())
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle forward of {rows.size} query rows (every {stride}th) of head (0,0) of the "
+                      f"workload, {dt:.1f} s; FLOPs counted as 4*d per visible key",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    import numpy as np
+
+    from oracle import oracle as OR
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = WORKLOAD
+    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
+    q, k, v, rows, stride, threads = _oracle_sample(per_step)
+    vis = (rows + 1) if w["causal"] else np.full(rows.shape, w["N"])
+    fl = float(4.0 * w["d"] * vis.sum())
+    for _ in range(args.warmup):
+        OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
+    dt = (time.perf_counter() - t) / max(1, args.steps)
+    value = fl / dt / 1e12
+    sample = (f"fp64 oracle forward of {rows.size} query rows (every {stride}th) of head (0,0) per step; "
+              f"FLOPs counted as 4*d per visible key")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": config_dict(world),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,114 @@
+"""Thin Python binding over the C ABI (include/fa.h), same names.
+
+Argument marshalling only: torch tensors (device memory) are turned into
+pointers and sizes and passed to libfa.so on the current CUDA stream.  Every
+computation runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import check
+
+_BF16 = torch.bfloat16
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
+                         f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} cuda={t.is_cuda}")
+
+
+def fa_fwd(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v); q/k/v bf16 [B, H, N, d] on the GPU."""
+    B, H, N, d = _shape(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, nm, _BF16, (B, H, N, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", _BF16, (B, H, N, d))
+    _need(lse, "lse", torch.float32, (B, H, N))
+    check(_lib.lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, scale,
+                            int(bool(causal)), _stream(stream)), "fa_fwd")
+    return out, lse
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.lib().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_bwd(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False,
+           dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of attention given the forward's O and LSE and the upstream dO."""
+    B, H, N, d = _shape(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, nm, _BF16, (B, H, N, d))
+    _need(lse, "lse", torch.float32, (B, H, N))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    ws_bytes = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, nm, _BF16, (B, H, N, d))
+    check(_lib.lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                            _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            B, H, N, d, scale, int(bool(causal)), _stream(stream)), "fa_bwd")
+    return dq, dk, dv
+
+
+def fa_last_device_status(stream=None) -> tuple[int, int]:
+    """(status, detail) after synchronising the stream; see include/fa.h."""
+    detail = ctypes.c_int(0)
+    rc = _lib.lib().fa_last_device_status(_stream(stream), ctypes.byref(detail))
+    return int(rc), int(detail.value)
+
+
+def fa_set_softmax_options(tau: float = 8.0, poly: int = 1) -> None:
+    check(_lib.lib().fa_set_softmax_options(float(tau), int(poly)), "fa_set_softmax_options")
+
+
+def fa_exp2_eval(x: torch.Tensor, mode: int = 0, stream=None) -> torch.Tensor:
+    """2^x on the device: mode 0 = cubic software exp2, 1 = SFU ex2."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    check(_lib.lib().fa_exp2_eval(_ptr(x), _ptr(y), x.numel(), int(mode), _stream(stream)), "fa_exp2_eval")
+    return y
+
+
+def fa_profile_next(which: int, start, stop) -> None:
+    """Have the next fa_fwd (0) / fa_bwd (1) record torch.cuda.Events around its main kernel."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event)
+    check(_lib.lib().fa_profile_next(int(which), h(start), h(stop)), "fa_profile_next")
+
+
+def fa_strerror(code: int) -> str:
+    return _lib.lib().fa_strerror(int(code)).decode()
+
+
+def fa_version() -> int:
+    return int(_lib.lib().fa_version())

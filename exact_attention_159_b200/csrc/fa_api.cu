@@ -1,0 +1,356 @@
+// fa_api.cu -- host side of libfa: argument checks, TMA descriptors, launches.
+// See include/fa.h for the contract of every entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "exp2_poly.cuh"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kPoly16 = 4;  // exponentials per 16 evaluated by the cubic when the polynomial path is on
+
+__device__ int g_status;  // first device-side failure (wait site), 0 = none
+
+struct DeviceState {
+  std::once_flag once;
+  int* status = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+
+float g_tau = fa::kRescaleTau;
+int g_poly = 1;
+cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // one-shot [fwd|bwd][start|stop]
+
+// Records the pending start event of `which` (if any) on `st`; returns whether one was pending.
+bool prof_begin(int which, cudaStream_t st) {
+  if (!g_prof[which][0]) return false;
+  cudaEventRecord(g_prof[which][0], st);
+  return true;
+}
+void prof_end(int which, cudaStream_t st) {
+  if (g_prof[which][1]) cudaEventRecord(g_prof[which][1], st);
+  g_prof[which][0] = g_prof[which][1] = nullptr;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Status word of the current device (set up once per device).
+int* device_status(int* err_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *err_out = FA_ERR_CUDA;
+    return nullptr;
+  }
+  DeviceState& s = g_dev[dev];
+  std::call_once(s.once, [&s] {
+    void* p = nullptr;
+    s.err = cudaGetSymbolAddress(&p, g_status);
+    if (s.err == cudaSuccess) s.status = static_cast<int*>(p);
+  });
+  if (!s.status) *err_out = FA_ERR_CUDA;
+  return s.status;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// 3-D map over a contiguous [BH, N, d] bf16 tensor: box 64 (d) x 128 (rows) x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Shape checks shared by forward and backward.  Returns FA_OK, or the error; *empty set for 0-size problems.
+int check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  const long long BH = static_cast<long long>(B) * H;
+  const long long tiles = (static_cast<long long>(N) + 127) / 128;
+  // grid size, tensor-map extents and int row indices must stay in range
+  if (BH > INT_MAX / 2 || BH * tiles > INT_MAX || static_cast<long long>(N) + 128 > INT_MAX) return FA_ERR_UNSUPPORTED;
+  if (BH * (tiles * 128) * d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, bool C, int P>
+int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const fa::FwdParams& prm,
+               cudaStream_t st) {
+  using L = fa::FwdLayout<D>;
+  auto kern = fa::fwd_kernel<D, C, P>;
+  if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_pairs);
+  kern<<<grid, L::kThreads, L::kBytes, st>>>(q, k, v, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool C>
+int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
+               const fa::BwdParams& prm, cudaStream_t st) {
+  using L = fa::BwdLayout<D>;
+  auto kern = fa::bwd_kernel<D, C>;
+  if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
+  kern<<<grid, 320, L::kBytes, st>>>(q, k, v, dO, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+struct WsLayout {
+  size_t dq, lse2, dsum, total;
+};
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+WsLayout ws_layout(long long BH, int N, int d) {
+  const size_t npad = static_cast<size_t>((N + 127) / 128) * 128;
+  WsLayout w;
+  w.dq = 0;
+  w.lse2 = round256(static_cast<size_t>(BH) * npad * d * sizeof(float));
+  w.dsum = w.lse2 + round256(static_cast<size_t>(BH) * npad * sizeof(float));
+  w.total = w.dsum + round256(static_cast<size_t>(BH) * npad * sizeof(float));
+  return w;
+}
+
+__global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int mode) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = mode == 0 ? fa::exp2_poly(x[i]) : fa::exp2_sfu(x[i]);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char* fa_strerror(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape or head dimension";
+    case FA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fa_set_softmax_options(float tau, int poly) {
+  if (!(tau >= 0.0f && tau <= 16.0f) || (poly != 0 && poly != 1)) return FA_ERR_INVALID_ARG;
+  g_tau = tau;
+  g_poly = poly;
+  return FA_OK;
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           float scale, int causal, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, H, N, d, scale, causal, &empty);
+  if (rc != FA_OK) return rc;
+  if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_ALIGNMENT;
+  const int BH = B * H;
+  const size_t nb = static_cast<size_t>(BH) * N * d * 2, lb = static_cast<size_t>(BH) * N * 4;
+  for (const void* in : {Q, K, V})
+    if (overlaps(O, nb, in, nb) || overlaps(LSE, lb, in, nb)) return FA_ERR_INVALID_ARG;
+  if (overlaps(O, nb, LSE, lb)) return FA_ERR_INVALID_ARG;
+  int* status = device_status(&rc);
+  if (!status) return rc;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d))
+    return FA_ERR_CUDA;
+  fa::FwdParams prm;
+  prm.O = static_cast<__nv_bfloat16*>(O);
+  prm.LSE = LSE;
+  prm.N = N;
+  prm.BH = BH;
+  const int tiles = (N + 127) / 128;
+  prm.n_pairs = (tiles + 1) / 2;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.tau = g_tau;
+  prm.status = status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool poly = g_poly != 0;
+  const bool prof = prof_begin(0, st);
+  if (d == 128) {
+    if (causal)
+      rc = poly ? launch_fwd<128, true, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<128, true, 0>(mq, mk, mv, prm, st);
+    else
+      rc = poly ? launch_fwd<128, false, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<128, false, 0>(mq, mk, mv, prm, st);
+  } else {
+    if (causal)
+      rc = poly ? launch_fwd<64, true, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<64, true, 0>(mq, mk, mv, prm, st);
+    else
+      rc = poly ? launch_fwd<64, false, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<64, false, 0>(mq, mk, mv, prm, st);
+  }
+  if (prof) prof_end(0, st);
+  return rc;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  bool empty = false;
+  if (check_shape(B, H, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  return ws_layout(static_cast<long long>(B) * H, N, d).total;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+           int causal, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, H, N, d, scale, causal, &empty);
+  if (rc != FA_OK) return rc;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  for (const void* p : {Q, K, V, O, dO, static_cast<const void*>(LSE), static_cast<const void*>(dQ),
+                        static_cast<const void*>(dK), static_cast<const void*>(dV), static_cast<const void*>(workspace)})
+    if (!aligned16(p)) return FA_ERR_ALIGNMENT;
+  const int BH = B * H;
+  const WsLayout ws = ws_layout(BH, N, d);
+  if (workspace_bytes < ws.total) return FA_ERR_INVALID_ARG;
+  const size_t nb = static_cast<size_t>(BH) * N * d * 2, lb = static_cast<size_t>(BH) * N * 4;
+  const void* outs[4] = {dQ, dK, dV, workspace};
+  const size_t osz[4] = {nb, nb, nb, ws.total};
+  const void* ins[6] = {Q, K, V, O, dO, LSE};
+  const size_t isz[6] = {nb, nb, nb, nb, nb, lb};
+  for (int a = 0; a < 4; ++a) {
+    for (int b = 0; b < 6; ++b)
+      if (overlaps(outs[a], osz[a], ins[b], isz[b])) return FA_ERR_INVALID_ARG;
+    for (int b = a + 1; b < 4; ++b)
+      if (overlaps(outs[a], osz[a], outs[b], osz[b])) return FA_ERR_INVALID_ARG;
+  }
+  int* status = device_status(&rc);
+  if (!status) return rc;
+
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d) ||
+      !make_map(&mdo, dO, BH, N, d))
+    return FA_ERR_CUDA;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  const int tiles = (N + 127) / 128;
+  const int npad = tiles * 128;
+  fa::BwdParams prm;
+  prm.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  prm.dsum = reinterpret_cast<const float*>(wsb + ws.dsum);
+  prm.dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
+  prm.dK = static_cast<__nv_bfloat16*>(dK);
+  prm.dV = static_cast<__nv_bfloat16*>(dV);
+  prm.N = N;
+  prm.Npad = npad;
+  prm.BH = BH;
+  prm.n_tiles = tiles;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.scale = scale;
+  prm.status = status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  const long long prep_rows = static_cast<long long>(BH) * npad;
+  const long long prep_threads = prep_rows * (d / 8);
+  const unsigned prep_grid = static_cast<unsigned>((prep_threads + 255) / 256);
+  float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
+  float* dsum = reinterpret_cast<float*>(wsb + ws.dsum);
+  if (d == 128)
+    fa::bwd_prep_kernel<128><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
+                                                        static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
+                                                        prm.dq_acc, N, npad, prep_rows);
+  else
+    fa::bwd_prep_kernel<64><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
+                                                       static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
+                                                       prm.dq_acc, N, npad, prep_rows);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  const bool prof = prof_begin(1, st);
+  if (d == 128)
+    rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, prm, st) : launch_bwd<128, false>(mq, mk, mv, mdo, prm, st);
+  else
+    rc = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, prm, st) : launch_bwd<64, false>(mq, mk, mv, mdo, prm, st);
+  if (prof) prof_end(1, st);
+  if (rc != FA_OK) return rc;
+
+  const long long rows = static_cast<long long>(BH) * N;
+  const unsigned cgrid = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
+  if (d == 128)
+    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(prm.dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+  else
+    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(prm.dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_last_device_status(void* stream, int* detail) {
+  if (detail) *detail = 0;
+  int rc = FA_OK;
+  int* status = device_status(&rc);
+  if (!status) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+    if (detail) *detail = v;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+int fa_profile_next(int which, void* start_event, void* stop_event) {
+  if ((which != 0 && which != 1) || (!start_event) != (!stop_event)) return FA_ERR_INVALID_ARG;
+  g_prof[which][0] = static_cast<cudaEvent_t>(start_event);
+  g_prof[which][1] = static_cast<cudaEvent_t>(stop_event);
+  return FA_OK;
+}
+
+int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream) {
+  if (!x || !y || n < 0 || (mode != 0 && mode != 1)) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return FA_ERR_ALIGNMENT;
+  if (n == 0) return FA_OK;
+  if (n > (1LL << 36)) return FA_ERR_UNSUPPORTED;
+  const unsigned grid = static_cast<unsigned>((n + 255) / 256);
+  exp2_eval_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, mode);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,415 @@
+// fa_bwd.cuh -- backward exact attention on sm_100a.
+//
+// P is recomputed from the saved log-sum-exp instead of being stored
+// (FlashAttention-4 pages: backward pass with intermediates kept in TMEM,
+// "using TMEM to store backward intermediates instead of SMEM").  Three
+// kernels run on the caller's stream:
+//   bwd_prep_kernel    D_i = dO_i . O_i, LSE2_i = LSE_i * log2(e) (+inf on the
+//                      padding rows of the last tile), dQ_acc = 0
+//   bwd_kernel         one CTA per (batch*head, 128-row key tile n), key tile
+//                      stationary, loop over the query tiles m that see it:
+//                        S^T  = K_n Q_m^T                 (tcgen05 -> TMEM)
+//                        P^T  = 2^(S^T scale log2e - LSE2) (CUDA cores -> TMEM, bf16)
+//                        dP^T = V_n dO_m^T                (tcgen05 -> TMEM)
+//                        dS^T = P^T (dP^T - D)            (CUDA cores -> smem, bf16)
+//                        dV  += P^T dO_m                  (A from TMEM)
+//                        dK  += dS^T Q_m
+//                        dQ_m = dS K_n                    (TMEM) -> fp32 atomics into dQ_acc
+//                      dK (x scale) and dV leave TMEM once, at the end.
+//   bwd_dq_kernel      dQ = bf16(scale * dQ_acc)
+// Warps: 0 TMA producer, 1 MMA issuer + TMEM owner, 2..5 P/dS for the 128 key
+// rows (thread = key row), 6..9 dQ drain (thread = query row).
+// Tensor memory columns: dK [0,D), dV [D,2D), S^T [2D,2D+128),
+// dP^T [2D+128,2D+256); dQ reuses the dP^T columns when D = 128 (the 512
+// columns are otherwise full) and has its own 64 columns when D = 64.
+#pragma once
+
+#include "fa_fwd.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const float* lse2;   // [BH, Npad]  LSE * log2(e), +inf on padding rows
+  const float* dsum;   // [BH, Npad]  D_i
+  float* dq_acc;       // [BH, Npad, D] fp32
+  __nv_bfloat16* dK;   // [BH, N, D]
+  __nv_bfloat16* dV;   // [BH, N, D]
+  int N, Npad, BH, n_tiles;
+  float scale_log2;    // scale * log2(e)
+  float scale;
+  int* status;
+};
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTileBytes;
+  static constexpr int kQ = kV + kTileBytes;
+  static constexpr int kdO = kQ + kTileBytes;
+  static constexpr int kdS = kdO + kTileBytes;     // dS^T, 128 x 128 bf16, two 64-column chunks
+  static constexpr int kLse = kdS + 32768;         // 128 fp32
+  static constexpr int kDsum = kLse + 512;         // 128 fp32
+  static constexpr int kBar = kDsum + 512;
+  // kv_full, q_full, q_empty, s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_free, acc_full, drain
+  static constexpr int kNumBars = 12;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kNeed = kMisc + 16 + 1024;
+  // Keep one CTA per SM (each CTA allocates all 512 TMEM columns).
+  static constexpr int kBytes = kNeed > 120 * 1024 ? kNeed : 120 * 1024;
+  static constexpr bool kAliasDQ = (D == 128);
+  static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 128;
+  static constexpr uint32_t kColDQ = kAliasDQ ? kColDP : 2 * D + 256;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+               const BwdParams prm) {
+  using L = BwdLayout<D>;
+  constexpr int T = L::kTileBytes;
+  constexpr int kChunks = D / 64;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t *kv_full = bars + 0, *q_full = bars + 1, *q_empty = bars + 2, *s_full = bars + 3;
+  uint64_t *dp_full = bars + 4, *p_full = bars + 5, *ds_full = bars + 6, *ds_empty = bars + 7;
+  uint64_t *dq_full = bars + 8, *dq_free = bars + 9, *acc_full = bars + 10, *drain = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
+  const float* sLse = reinterpret_cast<const float*>(smem + L::kLse);
+  const float* sDsum = reinterpret_cast<const float*>(smem + L::kDsum);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % prm.BH;
+  const int n = blockIdx.x / prm.BH;          // key tile; n = 0 has the most causal work
+  const int m_begin = CAUSAL ? n : 0;
+  const int n_m = prm.n_tiles - m_begin;      // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
+    mbar_init(ds_empty, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Guard g{abort_flag, prm.status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmdO);
+      mbar_expect_tx(kv_full, 2 * T);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(smem + L::kK + c * 16384, &tmK, 64 * c, n * kTile, bh, kv_full);
+        tma_load_3d(smem + L::kV + c * 16384, &tmV, 64 * c, n * kTile, bh, kv_full);
+      }
+      bool ok = true;
+      int issued = 0;
+      for (int mi = 0; mi < n_m; ++mi) {
+        const int m = m_begin + mi;
+        if (!(ok = wait(q_empty, (mi & 1) ^ 1, g, kSiteBwd | 1))) break;
+        mbar_expect_tx(q_full, 2 * T + 1024);
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(smem + L::kQ + c * 16384, &tmQ, 64 * c, m * kTile, bh, q_full);
+          tma_load_3d(smem + L::kdO + c * 16384, &tmdO, 64 * c, m * kTile, bh, q_full);
+        }
+        const size_t off = static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile;
+        bulk_load(smem + L::kLse, prm.lse2 + off, 512, q_full);
+        bulk_load(smem + L::kDsum, prm.dsum + off, 512, q_full);
+        ++issued;
+      }
+      if (!ok) {
+        drain_wait(kv_full, 0);
+        if (issued > 0) drain_wait(q_full, (issued - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: both K-major
+      constexpr uint32_t idKM = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK: B MN-major
+      constexpr uint32_t idMM = idesc_bf16_f32(128, D, true, true);      // dQ: A and B MN-major
+      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO);
+      const uint32_t sdS = smem_u32(smem + L::kdS);
+      bool ok = wait(kv_full, 0, g, kSiteBwd | 2);
+      for (int mi = 0; ok && mi < n_m; ++mi) {
+        const uint32_t ph = mi & 1;
+        if (!(ok = wait(q_full, ph, g, kSiteBwd | 3))) break;
+        tc_fence_after();
+        // S^T = K Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + L::kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idKK, kk > 0);
+        }
+        tc_commit(s_full);
+        // dP^T = V dO^T (its columns hold dQ of the previous tile when aliased)
+        if (L::kAliasDQ && mi > 0) {
+          if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 4))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + L::kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024), idKK,
+                 kk > 0);
+        }
+        tc_commit(dp_full);
+        // dV += P^T dO
+        if (!(ok = wait(p_full, ph, g, kSiteBwd | 5))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + L::kColDV, tmem + L::kColS + 8 * kk, sdesc_sw128(sdO + kk * 2048, 16384, 1024), idKM,
+                 (mi > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q
+        if (!(ok = wait(ds_full, ph, g, kSiteBwd | 6))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
+                 idKM, (mi > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(q_empty);  // Q_m, dO_m, LSE2_m, D_m no longer needed once these land
+        // dQ_m = dS K
+        if (!L::kAliasDQ && mi > 0) {
+          if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 7))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ss(tmem + L::kColDQ, sdesc_sw128(sdS + kk * 2048, 16384, 1024),
+                 sdesc_sw128(sK + kk * 2048, 16384, 1024), idMM, kk > 0);
+        tc_commit(dq_full);
+        tc_commit(ds_empty);
+      }
+      if (ok) tc_commit(acc_full);
+      tc_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else if (warp < 6) {
+    // --------------------------------------------------- P^T and dS^T rows
+    const int quarter = warp & 3;
+    const int j = quarter * 32 + lane;  // key row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + L::kColS + lane_off, tdP = tmem + L::kColDP + lane_off;
+    uint8_t* sdS = smem + L::kdS;
+    const float sl2 = prm.scale_log2;
+    bool ok = true;
+    for (int mi = 0; mi < n_m; ++mi) {
+      const int m = m_begin + mi;
+      const uint32_t ph = mi & 1;
+      // LSE2_m / D_m arrive with Q_m (TMA); S^T_m is ready once s_full completes
+      if (!(ok = wait_warp(q_full, ph, g, kSiteBwd | 13))) break;
+      if (!(ok = wait_warp(s_full, ph, g, kSiteBwd | 8))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+      float p[kTile];
+      const bool diag = CAUSAL && m == n;
+#pragma unroll
+      for (int i = 0; i < kTile; ++i) {
+        const float x = fmaf(__uint_as_float(sr[i >> 5][i & 31]), sl2, -sLse[i]);
+        p[i] = (diag && i < j) ? 0.0f : exp2_sfu(x);
+      }
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int i = 0; i < kTile; i += 2) pk[i >> 6][(i & 63) >> 1] = pack_bf16x2(p[i], p[i + 1]);
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+
+      if (!(ok = wait_warp(dp_full, ph, g, kSiteBwd | 9))) break;
+      tc_fence_after();
+      if (mi > 0) {
+        if (!(ok = wait_warp(ds_empty, ph ^ 1, g, kSiteBwd | 10))) break;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dp[32];
+        tmem_ld32(tdP + 32 * c, dp);
+        tmem_wait_ld();
+        reg_fence(dp);
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int i = 32 * c + e;
+          const float ds0 = p[i] * (__uint_as_float(dp[e]) - sDsum[i]);
+          const float ds1 = p[i + 1] * (__uint_as_float(dp[e + 1]) - sDsum[i + 1]);
+          w[e >> 1] = pack_bf16x2(ds0, ds1);
+        }
+        // columns 32c .. 32c+31 live in chunk (32c / 64), 16-byte groups 4*(c&1) .. +3
+        uint8_t* base = sdS + (c >> 1) * 16384;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t col = (c & 1) * 32 + q4 * 8;
+          *reinterpret_cast<uint4*>(base + sw128_offset(j, col)) =
+              make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok) ok = wait_warp(acc_full, 0, g, kSiteBwd | 11);
+    if (ok) {
+      tc_fence_after();
+      const int key = n * kTile + j;
+      const bool store = key < prm.N;
+      const size_t rowoff = (static_cast<size_t>(bh) * prm.N + (store ? key : 0)) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = tmem + (which == 0 ? L::kColDK : L::kColDV) + lane_off;
+        const float mul = which == 0 ? prm.scale : 1.0f;
+        __nv_bfloat16* dst_row = (which == 0 ? prm.dK : prm.dV) + rowoff;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tcol + 32 * c, a);
+          tmem_wait_ld();
+          reg_fence(a);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- dQ drain
+    const int quarter = warp & 3;
+    const int i = quarter * 32 + lane;  // query row within the tile
+    const uint32_t tdQ = tmem + L::kColDQ + (static_cast<uint32_t>(quarter * 32) << 16);
+    for (int mi = 0; mi < n_m; ++mi) {
+      const int m = m_begin + mi;
+      if (!wait_warp(dq_full, mi & 1, g, kSiteBwd | 12)) break;
+      tc_fence_after();
+      float4* acc = reinterpret_cast<float4*>(
+          prm.dq_acc + (static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile + i) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tdQ + 32 * c, a);
+        tmem_wait_ld();
+        reg_fence(a);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          atomicAdd(acc + 8 * c + v, make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                                 __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3])));
+      }
+      tc_fence_before();
+      mbar_arrive(dq_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D_i = sum_c dO_ic O_ic (fp32 from bf16), LSE2_i = LSE_i log2(e), dQ_acc = 0.
+// Rows i >= N of the padded last tile get D = 0 and LSE2 = +inf (so P = 0 there).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
+                                                       const __nv_bfloat16* __restrict__ dO,
+                                                       const float* __restrict__ LSE, float* __restrict__ lse2,
+                                                       float* __restrict__ dsum, float* __restrict__ dq_acc, int N,
+                                                       int Npad, long long rows_total) {
+  constexpr int G = D / 8;  // threads per row, 8 elements (16 bytes) each
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long r = t / G;
+  const int seg = static_cast<int>(t % G);
+  const bool live = r < rows_total;
+  const long long bh = live ? r / Npad : 0;
+  const int i = live ? static_cast<int>(r % Npad) : 0;
+  const bool valid = live && i < N;
+  float acc = 0.0f;
+  if (valid) {
+    const size_t e = (static_cast<size_t>(bh) * N + i) * D + seg * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(O + e);
+    const uint4 b = *reinterpret_cast<const uint4*>(dO + e);
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 fa = __bfloat1622float2(pa[k]), fb = __bfloat1622float2(pb[k]);
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (live) {
+    if (seg == 0) {
+      dsum[r] = valid ? acc : 0.0f;
+      lse2[r] = valid ? LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + r * D + seg * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dQ = bf16(scale * dQ_acc) for the N real rows of every head.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ dq_acc,
+                                                     __nv_bfloat16* __restrict__ dQ, float scale, int N, int Npad,
+                                                     long long rows_total) {
+  constexpr int G = D / 8;
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long r = t / G;  // over BH * N real rows
+  const int seg = static_cast<int>(t % G);
+  if (r >= rows_total) return;
+  const long long bh = r / N;
+  const int i = static_cast<int>(r % N);
+  const float4* src = reinterpret_cast<const float4*>(dq_acc + (bh * Npad + i) * D + seg * 8);
+  const float4 a = src[0], b = src[1];
+  uint4 o;
+  o.x = pack_bf16x2(a.x * scale, a.y * scale);
+  o.y = pack_bf16x2(a.z * scale, a.w * scale);
+  o.z = pack_bf16x2(b.x * scale, b.y * scale);
+  o.w = pack_bf16x2(b.z * scale, b.w * scale);
+  *reinterpret_cast<uint4*>(dQ + r * D + seg * 8) = o;
+}
+
+}  // namespace fa

@@ -1,0 +1,342 @@
+// fa_fwd.cuh -- forward exact attention on sm_100a (tcgen05 + TMEM + TMA).
+//
+// One CTA owns two 128-row query tiles of one (batch, head) ("ping-pong":
+// FlashAttention-4 pages, "A. La Danse du Ping-Pong" -- while the tensor core
+// works for one tile, the softmax warps work on the other).  Warp roles
+// ("The Technical Edge": warp specialisation into load / MMA / softmax /
+// output stages):
+//   warp 0      TMA producer: Q tiles once, then a ring of K/V tiles
+//   warp 1      MMA issuer (one thread) and TMEM owner
+//   warps 2..5  softmax + correction + epilogue for query tile 0
+//   warps 6..9  the same for query tile 1
+// Tensor memory (512 columns x 128 lanes x 32 bit, "TMEM (256 KB per SM)"):
+//   S_t = Q_t K^T  fp32, 128 columns at 128*t; P_t (bf16, packed two per
+//   column) is written back over the first 64 columns of S_t and read from
+//   there by the P.V MMA; O_t fp32, D columns at 256 + D*t.
+// Online softmax in base 2 with the running row maximum m (log2 units) and
+// conditional rescaling ("adaptive online softmax rescaling ... only when
+// maximum values change significantly"): O and l are rescaled only when the
+// tile maximum exceeds the reference maximum by more than tau = 8; otherwise
+// the stale reference is kept, so P <= 2^8.  The result is exact either way
+// because O / l and LSE use the same reference.
+// A fixed share of the exponentials of interior tiles runs as the cubic
+// polynomial on the FMA pipe, the rest on the SFU ("cubic polynomials ...
+// reduces SFU contention").
+#pragma once
+
+#include "exp2_poly.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kTile = 128;          // rows of a Q or K/V tile
+constexpr float kRescaleTau = 8.0f;  // log2 units
+
+// Error sites reported through the status word (low byte = kernel, next = site).
+enum : int { kSiteFwd = 0x100, kSiteBwd = 0x200 };
+
+struct FwdParams {
+  __nv_bfloat16* O;   // [BH, N, D]
+  float* LSE;         // [BH, N], natural log
+  int N;
+  int BH;
+  int n_pairs;        // ceil(ceil(N / 128) / 2)
+  float scale_log2;   // softmax scale * log2(e)
+  float tau;          // rescale threshold (log2 units)
+  int* status;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + 2 * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBar = kV + kStages * kTileBytes;
+  // q, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int kNumBars = 1 + 3 * kStages + 7;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16 + 1024;  // + alignment slack
+  static constexpr int kThreads = 320;
+};
+
+// Bounded wait that ignores the abort flag (used only to drain in-flight async work).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 200000000ull) break;
+  }
+}
+
+template <int D, bool CAUSAL, int POLY16>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
+  using L = FwdLayout<D>;
+  constexpr int S = L::kStages;
+  constexpr int T = L::kTileBytes;
+  constexpr int kChunks = D / 64;  // 128-byte swizzle chunks of 64 bf16 along d
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* bar_q = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + S;
+  uint64_t* kv_empty = v_full + S;
+  uint64_t* s_full = kv_empty + S;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % prm.BH;
+  const int pair = prm.n_pairs - 1 - blockIdx.x / prm.BH;  // heaviest causal work first
+  const int n_tiles = (prm.N + kTile - 1) / kTile;
+  int nkv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * pair + t;
+    nkv[t] = qt < n_tiles ? (CAUSAL ? qt + 1 : n_tiles) : 0;
+  }
+  const int nkv_max = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Guard g{abort_flag, prm.status};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_expect_tx(bar_q, (nkv[1] > 0 ? 2 : 1) * T);
+      for (int t = 0; t < 2; ++t)
+        if (nkv[t] > 0)
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(smem + L::kQ + t * T + c * 16384, &tmQ, 64 * c, (2 * pair + t) * kTile, bh, bar_q);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv_max; ++j) {
+        const int s = j % S;
+        const uint32_t ph = (j / S) & 1;
+        if (!(ok = wait(&kv_empty[s], ph ^ 1, g, kSiteFwd | 1))) break;
+        mbar_expect_tx(&k_full[s], T);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(smem + L::kK + s * T + c * 16384, &tmK, 64 * c, j * kTile, bh, &k_full[s]);
+        mbar_expect_tx(&v_full[s], T);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(smem + L::kV + s * T + c * 16384, &tmV, 64 * c, j * kTile, bh, &v_full[s]);
+        ++issued;
+      }
+      if (!ok) {  // let copies already in flight land before the CTA exits
+        drain_wait(bar_q, 0);
+        for (int i = issued - S > 0 ? issued - S : 0; i < issued; ++i) {
+          drain_wait(&k_full[i % S], (i / S) & 1);
+          drain_wait(&v_full[i % S], (i / S) & 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
+      const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+      auto issue_s = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + 128 * t, sdesc_sw128(sQ + t * T + off, 16, 1024), sdesc_sw128(sK + s * T + off, 16, 1024),
+                 idS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + 256 + D * t, tmem + 128 * t + 8 * kk, sdesc_sw128(sV + s * T + kk * 2048, 16384, 1024), idO,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait(bar_q, 0, g, kSiteFwd | 2) && wait(&k_full[0], 0, g, kSiteFwd | 3);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nkv[t] > 0) {
+            issue_s(t, 0);
+            tc_commit(&s_full[t]);
+          }
+      }
+      for (int j = 0; ok && j < nkv_max; ++j) {
+        const int s = j % S;
+        if (!(ok = wait(&v_full[s], (j / S) & 1, g, kSiteFwd | 4))) break;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          if (!(ok = wait(&p_full[t], j & 1, g, kSiteFwd | 5))) break;
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          tc_commit(&o_full[t]);
+          if (j + 1 < nkv[t]) {
+            const int s1 = (j + 1) % S;
+            if (!(ok = wait(&k_full[s1], ((j + 1) / S) & 1, g, kSiteFwd | 6))) break;
+            tc_fence_after();
+            issue_s(t, s1);
+            tc_commit(&s_full[t]);
+          }
+        }
+        if (ok) tc_commit(&kv_empty[s]);
+      }
+      tc_commit(drain);
+      drain_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------- softmax / correction / epilogue
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lanes this warp may touch: 32*quarter .. +31
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + 128 * t + lane_off;
+    const uint32_t tO = tmem + 256 + D * t + lane_off;
+    const int qt = 2 * pair + t;
+    const int row = qt * kTile + r;  // query row within the head
+    const float sl2 = prm.scale_log2;
+    float m_ref = -INFINITY, l = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nkv[t]; ++j) {
+      if (!(ok = wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+      float s[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+      const bool edge = (CAUSAL && j == qt) || ((j + 1) * kTile > prm.N);
+      if (edge) {
+        const int key0 = j * kTile;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) {
+          const int key = key0 + c;
+          if (key >= prm.N || (CAUSAL && key > row)) s[c] = -INFINITY;
+        }
+      }
+      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+      for (int c = 4; c < kTile; c += 4) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+        mx2 = fmaxf(mx2, s[c + 2]);
+        mx3 = fmaxf(mx3, s[c + 3]);
+      }
+      const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      const bool need = m_new > m_ref + prm.tau;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // correction: O_t *= 2^(m_ref - m_new) once the previous P.V has landed
+        if (!(ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8))) break;
+        tc_fence_after();
+        const float alpha = need ? exp2_sfu(m_ref - m_new) : 1.0f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      if (need) {
+        l *= exp2_sfu(m_ref - m_new);
+        m_ref = m_new;
+      }
+      const float neg_m = -m_ref;
+      float ls0 = 0.f, ls1 = 0.f;
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < kTile; c += 2) {
+        const float x0 = fmaf(s[c], sl2, neg_m), x1 = fmaf(s[c + 1], sl2, neg_m);
+        float p0, p1;
+        if (!edge && (c & 15) < POLY16) {
+          p0 = exp2_poly(x0);
+          p1 = exp2_poly(x1);
+        } else {
+          p0 = exp2_sfu(x0);
+          p1 = exp2_sfu(x1);
+        }
+        ls0 += p0;
+        ls1 += p1;
+        pk[c >> 6][(c & 63) >> 1] = pack_bf16x2(p0, p1);
+      }
+      l += ls0 + ls1;
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    if (ok && nkv[t] > 0) ok = wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
+    if (ok && nkv[t] > 0) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const bool store = row < prm.N;
+      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (store) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

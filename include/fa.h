@@ -1,0 +1,132 @@
+/*
+ * fa.h -- C ABI of libfa: exact scaled dot-product attention on one B200
+ * (sm_100a), forward and backward.
+ *
+ * The operation ("NVIDIA Blackwell: FlashAttention-4 Overcomes Memory
+ * Bottlenecks", body; "NVIDIA's FlashAttention-4: Cementing AI Infrastructure
+ * Dominance", "The Technical Edge"): for every (batch b, head h)
+ *
+ *     S    = scale * Q K^T,  with keys j > i masked out when causal
+ *            (queries and keys aligned at position 0)
+ *     LSE  = natural-log log-sum-exp of each row of S
+ *     O    = softmax(S) V = exp(S - LSE) V
+ *
+ * and the backward pass (recomputing P = exp(S - LSE) from the saved LSE):
+ *
+ *     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
+ *     dQ = scale * dS K,  dK = scale * dS^T Q.
+ *
+ * Layout: every tensor is contiguous [B, H, N, d] (d fastest), bf16 for
+ * Q, K, V, O, dO, dQ, dK, dV and fp32 for LSE ([B, H, N]).  All data
+ * pointers are DEVICE pointers; the caller owns every buffer.  The library
+ * allocates no device memory on any call; it keeps only a per-device status
+ * word and cached kernel attributes.
+ *
+ * Calls are asynchronous on the caller's stream (`stream` is a cudaStream_t,
+ * NULL = legacy default stream).  Argument checks happen on the host before
+ * anything is launched; a failing check returns its code and launches
+ * nothing.  No C++ exception crosses this interface and nothing calls exit.
+ *
+ * Supported: d in {64, 128}; any N >= 1 (a ragged last tile is masked);
+ * 0 < scale < inf.  Every pointer must be 16-byte aligned (TMA), and outputs
+ * must not overlap inputs.  Results are deterministic except dQ, whose fp32
+ * accumulation order (atomic adds across key tiles) varies between runs at
+ * the level of fp32 rounding.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad flag, bad scale, overlap */
+  FA_ERR_UNSUPPORTED = 2, /* head dim other than 64/128, sizes beyond the index range */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (launch, attributes, TMA encode) */
+  FA_ERR_TIMEOUT = 5      /* a kernel's bounded pipeline wait expired (see fa_last_device_status) */
+} fa_status;
+
+/*
+ * Forward.  Q, K, V: bf16 [B, H, N, d] (read).  O: bf16 [B, H, N, d]
+ * (written).  LSE: fp32 [B, H, N] (written), natural log: LSE_i =
+ * ln sum_j exp(S_ij).  B, H or N equal to 0 is an empty problem: returns
+ * FA_OK and launches nothing.  causal: 0 or 1.
+ * One kernel launch on `stream`.
+ */
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           float scale, int causal, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator
+ * [B, H, Npad, d] plus fp32 D and LSE*log2(e) vectors [B, H, Npad], with
+ * Npad = N rounded up to a multiple of 128, each part 256-byte aligned.
+ * Returns 0 for an empty or invalid shape.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward.  Q, K, V, O, dO: bf16 [B, H, N, d] (read); LSE: fp32 [B, H, N]
+ * as written by fa_fwd for the same Q, K, V, scale and causal (read).
+ * dQ, dK, dV: bf16 [B, H, N, d] (written).  workspace: device memory of at
+ * least fa_bwd_workspace_size() bytes, 16-byte aligned, owned by the caller;
+ * its contents on entry do not matter and it may be reused after the call's
+ * work on `stream` has finished.  Three kernel launches on `stream`
+ * (preprocess, main, dQ conversion).  Two fa_bwd calls that share a
+ * workspace must not overlap in time.
+ */
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+           void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+           float scale, int causal, void* stream);
+
+/* Static human-readable text for a status code. */
+const char* fa_strerror(int status);
+
+/*
+ * Synchronises `stream`, then reports device-side failures since the last
+ * call on the current device: FA_ERR_TIMEOUT if a kernel's bounded wait
+ * expired (the detail code, kernel and wait site, is returned through
+ * *detail when detail is not NULL), FA_ERR_CUDA if the synchronisation
+ * itself failed, FA_OK otherwise.  Clears the recorded failure.
+ */
+int fa_last_device_status(void* stream, int* detail);
+
+/*
+ * Tuning of the forward softmax (process-wide; for A/B comparisons).
+ * tau: rescale threshold in log2 units (0 <= tau <= 16; 0 = rescale whenever
+ * the running maximum grows).  poly: 1 = evaluate a quarter of the
+ * exponentials of interior tiles with the FMA-pipe cubic, 0 = all on the SFU.
+ * Returns FA_ERR_INVALID_ARG for values out of range.
+ */
+int fa_set_softmax_options(float tau, int poly);
+
+/*
+ * Elementwise y = 2^x on the device for testing the exponential the kernels
+ * use: mode 0 = the cubic-polynomial software exp2, mode 1 = the SFU
+ * (ex2.approx).  x, y: fp32 device arrays of n elements, 16-byte aligned.
+ */
+int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
+
+/*
+ * Profiling hook (used by the benchmark to time one kernel inside a call):
+ * when start_event and stop_event are cudaEvent_t handles, the NEXT fa_fwd
+ * (which = 0) or fa_bwd (which = 1) call records start_event on its stream
+ * immediately before its main attention kernel and stop_event immediately
+ * after it, then forgets both.  NULL, NULL clears a pending request.
+ * Returns FA_ERR_INVALID_ARG for another `which` or a half-NULL pair.
+ */
+int fa_profile_next(int which, void* start_event, void* stop_event);
+
+/* Library version, 100 * major + minor. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

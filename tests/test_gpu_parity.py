@@ -1,0 +1,183 @@
+"""GPU parity: libfa (through the C ABI) against the fp64 oracle on identical
+seeded bf16 inputs.
+
+Small shapes are compared element by element in full; the full-size workloads
+are compared on sampled rows (each query row of O / LSE / dQ, and each key row
+of dK / dV, is computable by the oracle on its own), plus invariants that hold
+at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_159_b200 import _lib, api, build
+from tests.gpu_util import TOL_GRAD, TOL_LSE, TOL_O, Case, bf16_to_f64, rel_l2, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    api.fa_set_softmax_options(8.0, 1)
+    yield
+    torch.cuda.synchronize()
+    assert api.fa_last_device_status() == (0, 0)
+
+
+def check_fwd(case, o, lse, heads, rows_per_head, label):
+    O_gpu = bf16_to_f64(o)
+    L_gpu = lse.cpu().numpy().astype(np.float64)
+    worst_o = worst_l = 0.0
+    for (b, h) in heads:
+        rows = None if rows_per_head is None else sample_rows(case.N, rows_per_head, 17 * b + h)
+        o_ref, l_ref = case.oracle_fwd(b, h, rows)
+        sel = np.arange(case.N) if rows is None else rows
+        worst_o = max(worst_o, float(np.abs(O_gpu[b, h][sel] - o_ref).max()))
+        worst_l = max(worst_l, float(np.abs(L_gpu[b, h][sel] - l_ref).max()))
+    print(f"[{label}] max|O-O_ref| = {worst_o:.3e}  max|LSE-LSE_ref| = {worst_l:.3e}")
+    assert worst_o <= TOL_O, f"{label}: O error {worst_o}"
+    assert worst_l <= TOL_LSE, f"{label}: LSE error {worst_l}"
+    return worst_o, worst_l
+
+
+def check_bwd(case, grads, heads, nq, nk, label):
+    dQ, dK, dV = (bf16_to_f64(g) for g in grads)
+    worst = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
+    for (b, h) in heads:
+        qr = None if nq is None else sample_rows(case.N, nq, 31 * b + h)
+        kr = None if nk is None else sample_rows(case.N, nk, 37 * b + h + 1)
+        dq, dk, dv, _, _ = case.oracle_bwd(b, h, qr, kr)
+        qs = np.arange(case.N) if qr is None else qr
+        ks = np.arange(case.N) if kr is None else kr
+        worst["dQ"] = max(worst["dQ"], rel_l2(dQ[b, h][qs], dq))
+        worst["dK"] = max(worst["dK"], rel_l2(dK[b, h][ks], dk))
+        worst["dV"] = max(worst["dV"], rel_l2(dV[b, h][ks], dv))
+    print(f"[{label}] rel L2: " + "  ".join(f"{k} {v:.3e}" for k, v in worst.items()))
+    for k, v in worst.items():
+        assert v <= TOL_GRAD, f"{label}: {k} relative L2 error {v}"
+    return worst
+
+
+def all_heads(case):
+    return [(b, h) for b in range(case.B) for h in range(case.H)]
+
+
+# ---------------------------------------------------------------- workloads
+def test_tiny_forward_and_backward_full():
+    c = Case(1, 1, 128, 64, False, seed_workload=1, bwd=True)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, [(0, 0)], None, "tiny fwd")
+    check_bwd(c, c.bwd_gpu(o, lse), [(0, 0)], None, None, "tiny bwd")
+
+
+def test_forward_causal_2048():
+    c = Case(4, 16, 2048, 128, True, seed_workload=2)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, all_heads(c), 160, "fwd causal B4 H16 N2048")
+
+
+def test_forward_rescale_stress_8192():
+    c = Case(2, 16, 8192, 128, False, seed_workload=3, stress=True)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, all_heads(c), 96, "fwd stress B2 H16 N8192")
+
+
+def test_long_context_forward_backward_32768():
+    c = Case(1, 16, 32768, 128, True, seed_workload=4, bwd=True)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, all_heads(c), 48, "fwd causal B1 H16 N32768")
+    grads = c.bwd_gpu(o, lse)
+    check_bwd(c, grads, [(0, 5)], 64, 64, "bwd causal B1 H16 N32768")
+    # invariants over every head: sum_j dV_j = sum_i dO_i, sum_j dK_j = 0
+    dK = bf16_to_f64(grads[1])
+    dV = bf16_to_f64(grads[2])
+    from exact_attention_159_b200 import inputs as I
+    dO = I.bf16_bits_to_f64(c.bits["do"])
+    for h in range(c.H):
+        s_dv, s_do = dV[0, h].sum(0), dO[0, h].sum(0)
+        assert rel_l2(s_dv, s_do) <= TOL_GRAD, f"head {h}: sum dV != sum dO"
+        spread = np.sqrt((np.linalg.norm(dK[0, h], axis=1) ** 2).sum())
+        assert np.linalg.norm(dK[0, h].sum(0)) <= 0.05 * spread, f"head {h}: sum dK != 0"
+
+
+SWEEP = [(B, N, d, causal) for (B, N) in ((8, 2048), (2, 8192), (1, 16384)) for d in (64, 128)
+         for causal in (False, True)]
+
+
+@pytest.mark.parametrize("B,N,d,causal", SWEEP, ids=[f"B{b}-N{n}-d{d}-{'c' if c else 'f'}" for b, n, d, c in SWEEP])
+def test_backward_sweep(B, N, d, causal):
+    c = Case(B, 16, N, d, causal, seed_workload=5, bwd=True)
+    o, lse = c.fwd_gpu()
+    heads = [(B - 1, 7)]
+    check_fwd(c, o, lse, heads, 48, f"sweep fwd B{B} N{N} d{d} causal={causal}")
+    check_bwd(c, c.bwd_gpu(o, lse), heads, 48, 48, f"sweep bwd B{B} N{N} d{d} causal={causal}")
+
+
+# --------------------------------------------------------------- edge cases
+EDGE = [(N, d, causal) for N in (1, 17, 127, 129, 200, 383) for d in (64, 128) for causal in (False, True)]
+
+
+@pytest.mark.parametrize("N,d,causal", EDGE, ids=[f"N{n}-d{d}-{'c' if c else 'f'}" for n, d, c in EDGE])
+def test_ragged_lengths_full(N, d, causal):
+    c = Case(1, 2, N, d, causal, seed_workload=11, bwd=True)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, all_heads(c), None, f"ragged N{N} d{d} c{int(causal)}")
+    check_bwd(c, c.bwd_gpu(o, lse), all_heads(c), None, None, f"ragged bwd N{N} d{d} c{int(causal)}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_several_tiles_and_heads_full(d, causal):
+    c = Case(2, 3, 640, d, causal, seed_workload=12, bwd=True)
+    o, lse = c.fwd_gpu()
+    check_fwd(c, o, lse, all_heads(c), None, f"multi d{d} c{int(causal)}")
+    check_bwd(c, c.bwd_gpu(o, lse), all_heads(c), None, None, f"multi bwd d{d} c{int(causal)}")
+
+
+@pytest.mark.parametrize("tau,poly", [(8.0, 1), (0.0, 0), (0.0, 1), (8.0, 0)])
+def test_rescale_and_exp_variants_agree(tau, poly):
+    c = Case(1, 4, 2048, 128, False, seed_workload=3, stress=True)
+    api.fa_set_softmax_options(8.0, 1)
+    o_ref_gpu, lse_ref_gpu = c.fwd_gpu()
+    try:
+        api.fa_set_softmax_options(tau, poly)
+        o, lse = c.fwd_gpu()
+    finally:
+        api.fa_set_softmax_options(8.0, 1)
+    check_fwd(c, o, lse, all_heads(c), 128, f"variant tau={tau} poly={poly}")
+    assert float((o.float() - o_ref_gpu.float()).abs().max()) <= TOL_O
+    assert float((lse - lse_ref_gpu).abs().max()) <= TOL_LSE
+
+
+def test_repeat_calls_deterministic():
+    c = Case(1, 4, 1024, 128, True, seed_workload=13, bwd=True)
+    o1, l1 = c.fwd_gpu()
+    o2, l2 = c.fwd_gpu()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    g1 = c.bwd_gpu(o1, l1)
+    g2 = c.bwd_gpu(o1, l1)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    # dQ accumulates with fp32 atomics in varying order: equal up to one bf16 ulp
+    assert float((g1[0].float() - g2[0].float()).abs().max()) <= 2.0 ** -6 * float(g1[0].float().abs().max())
+
+
+def test_empty_problem_is_noop():
+    lib = _lib.lib()
+    q = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    o = torch.full((16,), 7.0, dtype=torch.bfloat16, device="cuda")
+    l = torch.zeros(16, dtype=torch.float32, device="cuda")
+    import ctypes
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    assert lib.fa_fwd(P(q), P(q), P(q), P(o), P(l), 0, 4, 128, 64, 0.125, 0, None) == 0
+    torch.cuda.synchronize()
+    assert float(o.float().min()) == 7.0
+
+
+def test_unsupported_head_dim_launches_nothing():
+    q = torch.zeros((1, 1, 128, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.FAError) as e:
+        api.fa_fwd(q, q.clone(), q.clone())
+    assert e.value.code == _lib.FA_ERR_UNSUPPORTED
