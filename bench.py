@@ -335,6 +335,34 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_profile(args):
+    """A few plain calls on one shape, for ncu captures: --profile fwd|bwd --shape B,H,N,d."""
+    import numpy as np
+    import torch
+
+    from exact_attention_159_b200 import api, build, inputs as I
+
+    B, H, N, d = (int(x) for x in args.shape.split(","))
+    causal = bool(args.causal)
+    torch.cuda.set_device(0)
+    build.build()
+    bits = I.attention_inputs(4, B, H, N, d, with_do=True)
+    dev = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda() for k, v in bits.items()}
+    scale = 1.0 / math.sqrt(d)
+    o, lse = api.fa_fwd(dev["q"], dev["k"], dev["v"], scale, causal)
+    calls = 3
+    for _ in range(calls):
+        if args.profile == "fwd":
+            api.fa_fwd(dev["q"], dev["k"], dev["v"], scale, causal, out=o, lse=lse)
+        else:
+            api.fa_bwd(dev["q"], dev["k"], dev["v"], o, dev["do"], lse, scale, causal)
+    torch.cuda.synchronize()
+    rc, detail = api.fa_last_device_status()
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    print(f"profile {args.profile} B={B} H={H} N={N} d={d} causal={causal}: {calls + 1} calls ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,9 +371,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["fwd", "bwd"], help="plain calls on --shape for ncu captures")
+    ap.add_argument("--shape", default="1,16,16384,128", help="B,H,N,d for --profile")
+    ap.add_argument("--causal", type=int, default=1, help="causal flag for --profile")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
-    if args.impl == "reference":
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
