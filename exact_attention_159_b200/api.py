@@ -80,6 +80,23 @@ def fa_bwd(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False
     return dq, dk, dv
 
 
+def fa_bwd_noalloc(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False,
+                   dq=None, dk=None, dv=None, stream=None):
+    """fa_bwd on the library's fixed scratch array (no workspace; see include/fa.h for the size limit)."""
+    B, H, N, d = _shape(q)
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, nm, _BF16, (B, H, N, d))
+    _need(lse, "lse", torch.float32, (B, H, N))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    check(_lib.lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), B, H, N, d, scale, int(bool(causal)), _stream(stream)),
+          "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
 def fa_last_device_status(stream=None) -> tuple[int, int]:
     """(status, detail) after synchronising the stream; see include/fa.h."""
     detail = ctypes.c_int(0)

@@ -319,6 +319,54 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch for fa_bwd_noalloc: a fixed device array instead of a caller workspace.
+__device__ __align__(256) unsigned char g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+struct ScratchState {
+  std::once_flag once;
+  void* ptr = nullptr;
+};
+ScratchState g_scratch[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device;
+// in host code the symbol itself is only a host-side stand-in, never a device address).
+void* noalloc_scratch(int* err_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *err_out = FA_ERR_CUDA;
+    return nullptr;
+  }
+  ScratchState& s = g_scratch[dev];
+  std::call_once(s.once, [&s] {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) s.ptr = p;
+  });
+  if (!s.ptr) *err_out = FA_ERR_CUDA;
+  return s.ptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                   void* dQ, void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  const int rc0 = check_shape(B, H, N, d, scale, causal, &empty);
+  if (rc0 != FA_OK) return rc0;
+  if (!empty && fa_bwd_workspace_size(B, H, N, d) > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  int rc = FA_OK;
+  void* ws = noalloc_scratch(&rc);
+  if (!ws) return rc;
+  // fa_bwd's preprocess kernel rewrites D and LSE*log2(e) and zeroes the dQ accumulator on every call.
+  return fa_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, ws, FA_BWD_NOALLOC_SCRATCH_BYTES, B, H, N, d, scale, causal,
+                stream);
+}
+
 int fa_last_device_status(void* stream, int* detail) {
   if (detail) *detail = 0;
   int rc = FA_OK;

@@ -122,6 +122,38 @@ int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
  */
 int fa_profile_next(int which, void* start_event, void* stop_event);
 
+/* Size of the fixed device scratch array behind fa_bwd_noalloc (64 MiB). */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * fa_bwd_noalloc -- the backward pass for callers that cannot allocate
+ * device memory.  The paper has no counterpart; this entry point exists for
+ * integration only.  Some callers of this library cannot call cudaMalloc:
+ * for example a serving process whose memory manager has already reserved
+ * the whole device, or latency-critical code that must not pay for
+ * cudaMalloc's implicit device-wide synchronisation.  fa_bwd needs a caller
+ * workspace; this variant instead uses a scratch array of
+ * FA_BWD_NOALLOC_SCRATCH_BYTES that is a file-scope __device__ variable of
+ * the library, so every GPU that loads the library holds it until the
+ * process exits.  The caller still passes all inputs and outputs, with the
+ * same meaning, layout and checks as fa_bwd; nothing is allocated by the
+ * call (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * Limit: the problem must satisfy fa_bwd_workspace_size(B, H, N, d) <=
+ * FA_BWD_NOALLOC_SCRATCH_BYTES, i.e. B*H*ceil(N/128)*128 <= 129,024 rows at
+ * d = 128 (e.g. B*H = 16 heads of N = 8064) and <= 254,080 rows at d = 64;
+ * larger problems return FA_ERR_UNSUPPORTED before anything is launched.  The first call on a device looks up the scratch array's
+ * device address (cudaGetSymbolAddress, once per device, with that device
+ * current); make that first call before any stream capture.  Every call
+ * shares the one array and leaves its contents behind; each call clears
+ * what must start at zero itself.  Calls whose GPU work overlaps (different
+ * streams, or different host threads, on the same device) race on the
+ * scratch and give wrong results: serialise them.
+ */
+int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                   void* dQ, void* dK, void* dV, int B, int H, int N, int d, float scale, int causal,
+                   void* stream);
+
 /* Library version, 100 * major + minor. */
 int fa_version(void);
 
