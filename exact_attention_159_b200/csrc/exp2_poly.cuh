@@ -37,6 +37,23 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (ji << 23));
 }
 
+// exp2_poly on two values at once with packed fp32x2 arithmetic; the result is
+// bit for bit that of exp2_poly on each lane (every operation rounds the same
+// exact value: x - j is computed as fma(j, -1, x), and adding t << 23 to the
+// bits of p equals adding j << 23 because 0x4B400000 << 23 vanishes mod 2^32).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rd(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(FA_EXP2_C3, FA_EXP2_C3), f, make_float2(FA_EXP2_C2, FA_EXP2_C2));
+  p = __ffma2_rn(p, f, make_float2(FA_EXP2_C1, FA_EXP2_C1));
+  p = __ffma2_rn(p, f, make_float2(FA_EXP2_C0, FA_EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Hardware 2^x on the SFU (MUFU): ex2.approx, flush-to-zero; ex2(-inf) = +0.
 __device__ __forceinline__ float exp2_sfu(float x) {
   float y;

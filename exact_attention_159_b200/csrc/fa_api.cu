@@ -133,10 +133,10 @@ template <int D, bool C>
 int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
                const fa::BwdParams& prm, cudaStream_t st) {
   using L = fa::BwdLayout<D>;
-  auto kern = fa::bwd_kernel<D, C>;
+  auto kern = fa::bwd_kernel<D, C, kPoly16>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
-  kern<<<grid, 320, L::kBytes, st>>>(q, k, v, dO, prm);
+  kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -156,7 +156,14 @@ WsLayout ws_layout(long long BH, int N, int d) {
 
 __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int mode) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = mode == 0 ? fa::exp2_poly(x[i]) : fa::exp2_sfu(x[i]);
+  if (i >= n) return;
+  if (mode == 2) {  // packed form: lane i&1 of the pair (i & ~1, i | 1)
+    const long long i1 = (i | 1) < n ? (i | 1) : i;
+    const float2 r = fa::exp2_poly2(make_float2(x[i & ~1LL], x[i1]));
+    y[i] = (i & 1) ? r.y : r.x;
+  } else {
+    y[i] = mode == 0 ? fa::exp2_poly(x[i]) : fa::exp2_sfu(x[i]);
+  }
 }
 
 }  // namespace
@@ -273,8 +280,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   const int tiles = (N + 127) / 128;
   const int npad = tiles * 128;
   fa::BwdParams prm;
-  prm.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
-  prm.dsum = reinterpret_cast<const float*>(wsb + ws.dsum);
+  prm.nlse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  prm.ndsum = reinterpret_cast<const float*>(wsb + ws.dsum);
   prm.dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
   prm.dK = static_cast<__nv_bfloat16*>(dK);
   prm.dV = static_cast<__nv_bfloat16*>(dV);
@@ -392,7 +399,7 @@ int fa_profile_next(int which, void* start_event, void* stop_event) {
 }
 
 int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream) {
-  if (!x || !y || n < 0 || (mode != 0 && mode != 1)) return FA_ERR_INVALID_ARG;
+  if (!x || !y || n < 0 || mode < 0 || mode > 2) return FA_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return FA_ERR_ALIGNMENT;
   if (n == 0) return FA_OK;
   if (n > (1LL << 36)) return FA_ERR_UNSUPPORTED;

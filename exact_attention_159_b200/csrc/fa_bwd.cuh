@@ -29,8 +29,8 @@
 namespace fa {
 
 struct BwdParams {
-  const float* lse2;   // [BH, Npad]  LSE * log2(e), +inf on padding rows
-  const float* dsum;   // [BH, Npad]  D_i
+  const float* nlse2;  // [BH, Npad]  -LSE * log2(e), -inf on padding rows
+  const float* ndsum;  // [BH, Npad]  -D_i, 0 on padding rows
   float* dq_acc;       // [BH, Npad, D] fp32
   __nv_bfloat16* dK;   // [BH, N, D]
   __nv_bfloat16* dV;   // [BH, N, D]
@@ -45,16 +45,16 @@ struct BwdLayout {
   static constexpr int kTileBytes = kTile * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytes;
-  static constexpr int kQ = kV + kTileBytes;
-  static constexpr int kdO = kQ + kTileBytes;
-  static constexpr int kdS = kdO + kTileBytes;     // dS^T, 128 x 128 bf16, two 64-column chunks
-  static constexpr int kLse = kdS + 32768;         // 128 fp32
-  static constexpr int kDsum = kLse + 512;         // 128 fp32
-  static constexpr int kBar = kDsum + 512;
-  // kv_full, q_full, q_empty, s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_free, acc_full, drain
-  static constexpr int kNumBars = 12;
+  static constexpr int kQ = kV + kTileBytes;        // two stages
+  static constexpr int kdO = kQ + 2 * kTileBytes;   // two stages
+  static constexpr int kdS = kdO + 2 * kTileBytes;  // dS^T, 128 x 128 bf16, two 64-column chunks
+  static constexpr int kLse = kdS + 32768;          // two stages of 128 fp32 (-LSE2)
+  static constexpr int kDsum = kLse + 1024;         // two stages of 128 fp32 (-D)
+  static constexpr int kBar = kDsum + 1024;
+  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_free, acc_full, drain
+  static constexpr int kNumBars = 14;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kNeed = kMisc + 16 + 1024;
+  static constexpr int kNeed = kMisc + 16;           // the dynamic shared memory base is 1024-byte aligned
   // Keep one CTA per SM (each CTA allocates all 512 TMEM columns).
   static constexpr int kBytes = kNeed > 120 * 1024 ? kNeed : 120 * 1024;
   static constexpr bool kAliasDQ = (D == 128);
@@ -62,8 +62,12 @@ struct BwdLayout {
   static constexpr uint32_t kColDQ = kAliasDQ ? kColDP : 2 * D + 256;
 };
 
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+// Register split (setmaxnreg): 128 * (80 + 240 + 120) <= 384 * 168, the launch's total.  Each
+// setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
+constexpr int kBwdRegsCtl = 80, kBwdRegsP = 240, kBwdRegsDQ = 120;
+
+template <int D, bool CAUSAL, int POLY16>
+__global__ void __launch_bounds__(384, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const BwdParams prm) {
@@ -71,16 +75,17 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int T = L::kTileBytes;
   constexpr int kChunks = D / 64;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicCAS(prm.status, 0, kSiteBwd | 0x7F);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t *kv_full = bars + 0, *q_full = bars + 1, *q_empty = bars + 2, *s_full = bars + 3;
-  uint64_t *dp_full = bars + 4, *p_full = bars + 5, *ds_full = bars + 6, *ds_empty = bars + 7;
-  uint64_t *dq_full = bars + 8, *dq_free = bars + 9, *acc_full = bars + 10, *drain = bars + 11;
+  uint64_t *kv_full = bars + 0, *q_full = bars + 1, *q_empty = bars + 3, *s_full = bars + 5;
+  uint64_t *dp_full = bars + 6, *p_full = bars + 7, *ds_full = bars + 8, *ds_empty = bars + 9;
+  uint64_t *dq_full = bars + 10, *dq_free = bars + 11, *acc_full = bars + 12, *drain = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
-  const float* sLse = reinterpret_cast<const float*>(smem + L::kLse);
-  const float* sDsum = reinterpret_cast<const float*>(smem + L::kDsum);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x % prm.BH;
@@ -90,8 +95,10 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(&q_full[st], 1);
+      mbar_init(&q_empty[st], 1);
+    }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 128);
@@ -113,8 +120,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, prm.status};
-
-  if (warp == 0) {
+  if (warp < 4) {
+    regs_dec<kBwdRegsCtl>();
+    if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -129,36 +137,38 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       int issued = 0;
       for (int mi = 0; mi < n_m; ++mi) {
-        const int m = m_begin + mi;
-        if (!(ok = wait(q_empty, (mi & 1) ^ 1, g, kSiteBwd | 1))) break;
-        mbar_expect_tx(q_full, 2 * T + 1024);
+        const int m = m_begin + mi, st = mi & 1;
+        if (!(ok = wait(&q_empty[st], ((mi >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
+        mbar_expect_tx(&q_full[st], 2 * T + 1024);
         for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(smem + L::kQ + c * 16384, &tmQ, 64 * c, m * kTile, bh, q_full);
-          tma_load_3d(smem + L::kdO + c * 16384, &tmdO, 64 * c, m * kTile, bh, q_full);
+          tma_load_3d(smem + L::kQ + st * T + c * 16384, &tmQ, 64 * c, m * kTile, bh, &q_full[st]);
+          tma_load_3d(smem + L::kdO + st * T + c * 16384, &tmdO, 64 * c, m * kTile, bh, &q_full[st]);
         }
         const size_t off = static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile;
-        bulk_load(smem + L::kLse, prm.lse2 + off, 512, q_full);
-        bulk_load(smem + L::kDsum, prm.dsum + off, 512, q_full);
+        bulk_load(smem + L::kLse + 512 * st, prm.nlse2 + off, 512, &q_full[st]);
+        bulk_load(smem + L::kDsum + 512 * st, prm.ndsum + off, 512, &q_full[st]);
         ++issued;
       }
       if (!ok) {
         drain_wait(kv_full, 0);
-        if (issued > 0) drain_wait(q_full, (issued - 1) & 1);
+        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) drain_wait(&q_full[i & 1], (i >> 1) & 1);
       }
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: both K-major
       constexpr uint32_t idKM = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK: B MN-major
       constexpr uint32_t idMM = idesc_bf16_f32(128, D, true, true);      // dQ: A and B MN-major
       const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-      const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO);
+      const uint32_t sQ0 = smem_u32(smem + L::kQ), sdO0 = smem_u32(smem + L::kdO);
       const uint32_t sdS = smem_u32(smem + L::kdS);
       bool ok = wait(kv_full, 0, g, kSiteBwd | 2);
       for (int mi = 0; ok && mi < n_m; ++mi) {
+        const int st = mi & 1;
         const uint32_t ph = mi & 1;
-        if (!(ok = wait(q_full, ph, g, kSiteBwd | 3))) break;
+        const uint32_t sQ = sQ0 + st * T, sdO = sdO0 + st * T;
+        if (!(ok = wait(&q_full[st], (mi >> 1) & 1, g, kSiteBwd | 3))) break;
         tc_fence_after();
         // S^T = K Q^T
 #pragma unroll
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(320, 1)
           mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
                  idKM, (mi > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(q_empty);  // Q_m, dO_m, LSE2_m, D_m no longer needed once these land
+        tc_commit(&q_empty[st]);  // Q_m, dO_m, -LSE2_m, -D_m no longer needed once these land
         // dQ_m = dS K
         if (!L::kAliasDQ && mi > 0) {
           if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 7))) break;
@@ -212,20 +222,24 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit(drain);
       drain_wait(drain, 0);
     }
-  } else if (warp < 6) {
+    }
+  } else if (warp < 8) {
+    regs_inc<kBwdRegsP>();
     // --------------------------------------------------- P^T and dS^T rows
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // key row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + L::kColS + lane_off, tdP = tmem + L::kColDP + lane_off;
     uint8_t* sdS = smem + L::kdS;
-    const float sl2 = prm.scale_log2;
+    const float2 c2 = make_float2(prm.scale_log2, prm.scale_log2);
     bool ok = true;
     for (int mi = 0; mi < n_m; ++mi) {
-      const int m = m_begin + mi;
+      const int m = m_begin + mi, st = mi & 1;
       const uint32_t ph = mi & 1;
-      // LSE2_m / D_m arrive with Q_m (TMA); S^T_m is ready once s_full completes
-      if (!(ok = wait_warp(q_full, ph, g, kSiteBwd | 13))) break;
+      const float4* nl4 = reinterpret_cast<const float4*>(smem + L::kLse + 512 * st);
+      const float4* nd4 = reinterpret_cast<const float4*>(smem + L::kDsum + 512 * st);
+      // -LSE2_m / -D_m arrive with Q_m (TMA); S^T_m is ready once s_full completes
+      if (!(ok = wait_warp(&q_full[st], (mi >> 1) & 1, g, kSiteBwd | 13))) break;
       if (!(ok = wait_warp(s_full, ph, g, kSiteBwd | 8))) break;
       tc_fence_after();
       uint32_t sr[4][32];
@@ -236,16 +250,37 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
       float p[kTile];
       const bool diag = CAUSAL && m == n;
+      const bool edge = diag || (m + 1) * kTile > prm.N;
 #pragma unroll
-      for (int i = 0; i < kTile; ++i) {
-        const float x = fmaf(__uint_as_float(sr[i >> 5][i & 31]), sl2, -sLse[i]);
-        p[i] = (diag && i < j) ? 0.0f : exp2_sfu(x);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int i = 32 * cc + 4 * e4;
+          const float4 nl = nl4[i >> 2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int ii = i + 2 * h;
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[cc][ii & 31]), __uint_as_float(sr[cc][(ii + 1) & 31])),
+                                        c2, h == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
+            float2 pv;
+            if (!edge && ((ii >> 1) & 7) < POLY16 / 2) {
+              pv = exp2_poly2(x);
+            } else {
+              pv.x = exp2_sfu(x.x);
+              pv.y = exp2_sfu(x.y);
+              if (diag) {  // query i < key j is masked
+                if (ii < j) pv.x = 0.0f;
+                if (ii + 1 < j) pv.y = 0.0f;
+              }
+            }
+            p[ii] = pv.x;
+            p[ii + 1] = pv.y;
+            pk[(ii & 31) >> 1] = pack_bf16x2(pv.x, pv.y);
+          }
+        }
+        tmem_st16(tS + 16 * cc, pk);
       }
-      uint32_t pk[2][32];
-#pragma unroll
-      for (int i = 0; i < kTile; i += 2) pk[i >> 6][(i & 63) >> 1] = pack_bf16x2(p[i], p[i + 1]);
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -263,11 +298,17 @@ __global__ void __launch_bounds__(320, 1)
         reg_fence(dp);
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int i = 32 * c + e;
-          const float ds0 = p[i] * (__uint_as_float(dp[e]) - sDsum[i]);
-          const float ds1 = p[i + 1] * (__uint_as_float(dp[e + 1]) - sDsum[i + 1]);
-          w[e >> 1] = pack_bf16x2(ds0, ds1);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int i = 32 * c + 4 * e4;
+          const float4 nd = nd4[i >> 2];
+          const float2 t0 = __fadd2_rn(make_float2(__uint_as_float(dp[4 * e4]), __uint_as_float(dp[4 * e4 + 1])),
+                                       make_float2(nd.x, nd.y));
+          const float2 t1 = __fadd2_rn(make_float2(__uint_as_float(dp[4 * e4 + 2]), __uint_as_float(dp[4 * e4 + 3])),
+                                       make_float2(nd.z, nd.w));
+          const float2 d0 = __fmul2_rn(make_float2(p[i], p[i + 1]), t0);
+          const float2 d1 = __fmul2_rn(make_float2(p[i + 2], p[i + 3]), t1);
+          w[2 * e4] = pack_bf16x2(d0.x, d0.y);
+          w[2 * e4 + 1] = pack_bf16x2(d1.x, d1.y);
         }
         // columns 32c .. 32c+31 live in chunk (32c / 64), 16-byte groups 4*(c&1) .. +3
         uint8_t* base = sdS + (c >> 1) * 16384;
@@ -312,6 +353,7 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
+    regs_dec<kBwdRegsDQ>();
     // ----------------------------------------------------------- dQ drain
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;  // query row within the tile
@@ -347,13 +389,13 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-// D_i = sum_c dO_ic O_ic (fp32 from bf16), LSE2_i = LSE_i log2(e), dQ_acc = 0.
+// -D_i = -sum_c dO_ic O_ic (fp32 from bf16), -LSE2_i = -LSE_i log2(e), dQ_acc = 0.
 // Rows i >= N of the padded last tile get D = 0 and LSE2 = +inf (so P = 0 there).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ O,
                                                        const __nv_bfloat16* __restrict__ dO,
-                                                       const float* __restrict__ LSE, float* __restrict__ lse2,
-                                                       float* __restrict__ dsum, float* __restrict__ dq_acc, int N,
+                                                       const float* __restrict__ LSE, float* __restrict__ nlse2,
+                                                       float* __restrict__ ndsum, float* __restrict__ dq_acc, int N,
                                                        int Npad, long long rows_total) {
   constexpr int G = D / 8;  // threads per row, 8 elements (16 bytes) each
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -381,8 +423,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
   for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (live) {
     if (seg == 0) {
-      dsum[r] = valid ? acc : 0.0f;
-      lse2[r] = valid ? LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : INFINITY;
+      ndsum[r] = valid ? -acc : 0.0f;
+      nlse2[r] = valid ? -LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : -INFINITY;
     }
     float4* z = reinterpret_cast<float4*>(dq_acc + r * D + seg * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -7,8 +7,12 @@
 // output stages):
 //   warp 0      TMA producer: Q tiles once, then a ring of K/V tiles
 //   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 2..5  softmax + correction + epilogue for query tile 0
-//   warps 6..9  the same for query tile 1
+//   warps 2, 3  idle (they complete the first warpgroup)
+//   warps 4..7  softmax + correction + epilogue for query tile 0
+//   warps 8..11 the same for query tile 1
+// Registers are re-split per warpgroup with setmaxnreg (56 / 224 / 224 of
+// the 168 x 384 launched), so the softmax rows (128 fp32 scores each) stay in
+// registers.  The softmax arithmetic uses packed fp32x2 FMA/add.
 // Tensor memory (512 columns x 128 lanes x 32 bit, "TMEM (256 KB per SM)"):
 //   S_t = Q_t K^T  fp32, 128 columns at 128*t; P_t (bf16, packed two per
 //   column) is written back over the first 64 columns of S_t and read from
@@ -57,8 +61,8 @@ struct FwdLayout {
   // q, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
   static constexpr int kNumBars = 1 + 3 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 16 + 1024;  // + alignment slack
-  static constexpr int kThreads = 320;
+  static constexpr int kBytes = kMisc + 16;  // the dynamic shared memory base is 1024-byte aligned
+  static constexpr int kThreads = 384;
 };
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight async work).
@@ -69,8 +73,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Register split (setmaxnreg): 128 * (56 + 224 + 224) = 384 * 168, the launch's total.  Each
+// setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
+constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 224;
+
 template <int D, bool CAUSAL, int POLY16>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
   using L = FwdLayout<D>;
@@ -78,8 +86,11 @@ __global__ void __launch_bounds__(320, 1)
   constexpr int T = L::kTileBytes;
   constexpr int kChunks = D / 64;  // 128-byte swizzle chunks of 64 bf16 along d
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {  // swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicCAS(prm.status, 0, kSiteFwd | 0x7F);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* bar_q = bars;
   uint64_t* k_full = bars + 1;
@@ -129,8 +140,9 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, prm.status};
-
-  if (warp == 0) {
+  if (warp < 4) {
+    regs_dec<kFwdRegsCtl>();
+    if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
@@ -214,9 +226,11 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit(drain);
       drain_wait(drain, 0);
     }
+    }
   } else {
+    regs_inc<kFwdRegsSoftmax>();
     // ------------------------------------------- softmax / correction / epilogue
-    const int t = (warp - 2) >> 2;
+    const int t = (warp >> 2) - 1;
     const int quarter = warp & 3;  // TMEM lanes this warp may touch: 32*quarter .. +31
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -236,27 +250,26 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-      float s[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sr[c >> 5][c & 31]);
+      // scores stay in the registers tcgen05.ld wrote (S(c) reads column c as fp32)
+#define S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
       const bool edge = (CAUSAL && j == qt) || ((j + 1) * kTile > prm.N);
       if (edge) {
         const int key0 = j * kTile;
 #pragma unroll
         for (int c = 0; c < kTile; ++c) {
           const int key = key0 + c;
-          if (key >= prm.N || (CAUSAL && key > row)) s[c] = -INFINITY;
+          if (key >= prm.N || (CAUSAL && key > row)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
       }
-      float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+      // row maximum: four independent chains of 3-input max
+      float mx[4] = {S(0), S(32), S(64), S(96)};
 #pragma unroll
-      for (int c = 4; c < kTile; c += 4) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-        mx2 = fmaxf(mx2, s[c + 2]);
-        mx3 = fmaxf(mx3, s[c + 3]);
-      }
-      const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int c = 32 * q + 1; c < 32 * q + 31; c += 2) mx[q] = fmax3(mx[q], S(c), S(c + 1));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mx[q] = fmaxf(mx[q], S(32 * q + 31));
+      const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
       const bool need = m_new > m_ref + prm.tau;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // correction: O_t *= 2^(m_ref - m_new) once the previous P.V has landed
@@ -279,27 +292,34 @@ __global__ void __launch_bounds__(320, 1)
         l *= exp2_sfu(m_ref - m_new);
         m_ref = m_new;
       }
-      const float neg_m = -m_ref;
-      float ls0 = 0.f, ls1 = 0.f;
-      uint32_t pk[2][32];
+      // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 columns at a time)
+      const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
+      float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < kTile; c += 2) {
-        const float x0 = fmaf(s[c], sl2, neg_m), x1 = fmaf(s[c + 1], sl2, neg_m);
-        float p0, p1;
-        if (!edge && (c & 15) < POLY16) {
-          p0 = exp2_poly(x0);
-          p1 = exp2_poly(x1);
-        } else {
-          p0 = exp2_sfu(x0);
-          p1 = exp2_sfu(x1);
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = 32 * cc + 2 * e;
+          const float2 x = __ffma2_rn(make_float2(S(c), S(c + 1)), c2, nm2);
+          float2 p;
+          if (!edge && (e & 7) < POLY16 / 2) {
+            p = exp2_poly2(x);
+          } else {
+            p.x = exp2_sfu(x.x);
+            p.y = exp2_sfu(x.y);
+          }
+          if (e & 1)
+            ls1 = __fadd2_rn(ls1, p);
+          else
+            ls0 = __fadd2_rn(ls0, p);
+          pk[e] = pack_bf16x2(p.x, p.y);
         }
-        ls0 += p0;
-        ls1 += p1;
-        pk[c >> 6][(c & 63) >> 1] = pack_bf16x2(p0, p1);
+        tmem_st16(tS + 16 * cc, pk);
       }
-      l += ls0 + ls1;
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+#undef S
+      const float2 ls = __fadd2_rn(ls0, ls1);
+      l += ls.x + ls.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);

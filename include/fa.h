@@ -108,7 +108,9 @@ int fa_set_softmax_options(float tau, int poly);
 /*
  * Elementwise y = 2^x on the device for testing the exponential the kernels
  * use: mode 0 = the cubic-polynomial software exp2, mode 1 = the SFU
- * (ex2.approx).  x, y: fp32 device arrays of n elements, 16-byte aligned.
+ * (ex2.approx), mode 2 = the cubic with packed fp32x2 arithmetic on element
+ * pairs (must equal mode 0 bit for bit).  x, y: fp32 device arrays of n
+ * elements, 16-byte aligned.
  */
 int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
 

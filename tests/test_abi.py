@@ -119,6 +119,7 @@ def test_softmax_options_validation(lib):
 
 def test_exp2_eval_validation(lib):
     assert lib.fa_exp2_eval(P, P2, 10, 3, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_exp2_eval(P, P2, 10, -1, None) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_exp2_eval(MIS, P2, 10, 0, None) == _lib.FA_ERR_ALIGNMENT
     assert lib.fa_exp2_eval(P, P2, 0, 0, None) == _lib.FA_OK
 

@@ -35,3 +35,11 @@ def test_sfu_exp2_and_masked_input():
     assert rel.max() <= 1e-6
     z = api.fa_exp2_eval(torch.tensor([-np.inf, 0.0, 8.0, -200.0], dtype=torch.float32, device="cuda"), mode=1)
     assert z.cpu().tolist() == [0.0, 1.0, 256.0, 0.0]
+
+
+def test_packed_poly_equals_scalar_poly():
+    x = sweep_points(1 << 22)
+    xd = torch.from_numpy(x).cuda()
+    a = api.fa_exp2_eval(xd, mode=0).cpu().numpy()
+    b = api.fa_exp2_eval(xd, mode=2).cpu().numpy()
+    assert np.array_equal(a.view(np.int32), b.view(np.int32))
