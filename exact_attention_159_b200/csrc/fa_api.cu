@@ -94,6 +94,21 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the fp32 dQ accumulator [BH, Npad, d]: box 32 (d) x 128 (rows) x 1, 128-byte swizzle
+// (the layout of the backward kernel's staging buffers for its TMA reduce-add).
+bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(npad),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(npad) * d * 4};
+  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Shape checks shared by forward and backward.  Returns FA_OK, or the error; *empty set for 0-size problems.
 int check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
   *empty = false;
@@ -131,12 +146,12 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
 
 template <int D, bool C>
 int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
-               const fa::BwdParams& prm, cudaStream_t st) {
+               const CUtensorMap& dq_acc, const fa::BwdParams& prm, cudaStream_t st) {
   using L = fa::BwdLayout<D>;
   auto kern = fa::bwd_kernel<D, C, kPoly16>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
-  kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, prm);
+  kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -272,17 +287,17 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   int* status = device_status(&rc);
   if (!status) return rc;
 
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d) ||
-      !make_map(&mdo, dO, BH, N, d))
-    return FA_ERR_CUDA;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   const int tiles = (N + 127) / 128;
   const int npad = tiles * 128;
+  float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
+  CUtensorMap mq, mk, mv, mdo, macc;
+  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d) ||
+      !make_map(&mdo, dO, BH, N, d) || !make_acc_map(&macc, dq_acc, BH, npad, d))
+    return FA_ERR_CUDA;
   fa::BwdParams prm;
   prm.nlse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
   prm.ndsum = reinterpret_cast<const float*>(wsb + ws.dsum);
-  prm.dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
   prm.dK = static_cast<__nv_bfloat16*>(dK);
   prm.dV = static_cast<__nv_bfloat16*>(dV);
   prm.N = N;
@@ -302,27 +317,29 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   if (d == 128)
     fa::bwd_prep_kernel<128><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
                                                         static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                        prm.dq_acc, N, npad, prep_rows);
+                                                        dq_acc, N, npad, prep_rows);
   else
     fa::bwd_prep_kernel<64><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
                                                        static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                       prm.dq_acc, N, npad, prep_rows);
+                                                       dq_acc, N, npad, prep_rows);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   const bool prof = prof_begin(1, st);
   if (d == 128)
-    rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, prm, st) : launch_bwd<128, false>(mq, mk, mv, mdo, prm, st);
+    rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, macc, prm, st)
+                : launch_bwd<128, false>(mq, mk, mv, mdo, macc, prm, st);
   else
-    rc = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, prm, st) : launch_bwd<64, false>(mq, mk, mv, mdo, prm, st);
+    rc = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, macc, prm, st)
+                : launch_bwd<64, false>(mq, mk, mv, mdo, macc, prm, st);
   if (prof) prof_end(1, st);
   if (rc != FA_OK) return rc;
 
   const long long rows = static_cast<long long>(BH) * N;
   const unsigned cgrid = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
   if (d == 128)
-    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(prm.dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
   else
-    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(prm.dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -31,7 +31,6 @@ namespace fa {
 struct BwdParams {
   const float* nlse2;  // [BH, Npad]  -LSE * log2(e), -inf on padding rows
   const float* ndsum;  // [BH, Npad]  -D_i, 0 on padding rows
-  float* dq_acc;       // [BH, Npad, D] fp32
   __nv_bfloat16* dK;   // [BH, N, D]
   __nv_bfloat16* dV;   // [BH, N, D]
   int N, Npad, BH, n_tiles;
@@ -46,13 +45,15 @@ struct BwdLayout {
   static constexpr int kK = 0;
   static constexpr int kV = kK + kTileBytes;
   static constexpr int kQ = kV + kTileBytes;        // two stages
-  static constexpr int kdO = kQ + 2 * kTileBytes;   // two stages
-  static constexpr int kdS = kdO + 2 * kTileBytes;  // dS^T, 128 x 128 bf16, two 64-column chunks
-  static constexpr int kLse = kdS + 32768;          // two stages of 128 fp32 (-LSE2)
+  static constexpr int kdO = kQ + 2 * kTileBytes;   // one stage
+  static constexpr int kdS = kdO + kTileBytes;      // dS^T, 128 x 128 bf16, two 64-column chunks
+  static constexpr int kDQ = kdS + 32768;           // two 16 KB staging buffers: 128 rows x 32 fp32 of dQ
+  static constexpr int kLse = kDQ + 32768;          // two stages of 128 fp32 (-LSE2)
   static constexpr int kDsum = kLse + 1024;         // two stages of 128 fp32 (-D)
   static constexpr int kBar = kDsum + 1024;
-  // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_free, acc_full, drain
-  static constexpr int kNumBars = 14;
+  // kv_full, q_full[2], q_empty[2], do_full, do_empty, s_full, dp_full, p_full, ds_full, ds_empty,
+  // dq_full, dq_free, acc_full, drain
+  static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kNeed = kMisc + 16;           // the dynamic shared memory base is 1024-byte aligned
   // Keep one CTA per SM (each CTA allocates all 512 TMEM columns).
@@ -62,15 +63,15 @@ struct BwdLayout {
   static constexpr uint32_t kColDQ = kAliasDQ ? kColDP : 2 * D + 256;
 };
 
-// Register split (setmaxnreg): 128 * (80 + 240 + 120) <= 384 * 168, the launch's total.  Each
+// Register split (setmaxnreg): 128 * (80 + 240 + 184) = 384 * 168, the launch's total.  Each
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
-constexpr int kBwdRegsCtl = 80, kBwdRegsP = 240, kBwdRegsDQ = 120;
+constexpr int kBwdRegsCtl = 80, kBwdRegsP = 240, kBwdRegsDQ = 184;
 
 template <int D, bool CAUSAL, int POLY16>
 __global__ void __launch_bounds__(384, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-               const BwdParams prm) {
+               const __grid_constant__ CUtensorMap tmdQacc, const BwdParams prm) {
   using L = BwdLayout<D>;
   constexpr int T = L::kTileBytes;
   constexpr int kChunks = D / 64;
@@ -81,9 +82,10 @@ __global__ void __launch_bounds__(384, 1)
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t *kv_full = bars + 0, *q_full = bars + 1, *q_empty = bars + 3, *s_full = bars + 5;
-  uint64_t *dp_full = bars + 6, *p_full = bars + 7, *ds_full = bars + 8, *ds_empty = bars + 9;
-  uint64_t *dq_full = bars + 10, *dq_free = bars + 11, *acc_full = bars + 12, *drain = bars + 13;
+  uint64_t *kv_full = bars + 0, *q_full = bars + 1, *q_empty = bars + 3, *do_full = bars + 5;
+  uint64_t *do_empty = bars + 6, *s_full = bars + 7, *dp_full = bars + 8, *p_full = bars + 9;
+  uint64_t *ds_full = bars + 10, *ds_empty = bars + 11, *dq_full = bars + 12, *dq_free = bars + 13;
+  uint64_t *acc_full = bars + 14, *drain = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
 
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[st], 1);
       mbar_init(&q_empty[st], 1);
     }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 128);
@@ -120,108 +124,131 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, prm.status};
+
   if (warp < 4) {
     regs_dec<kBwdRegsCtl>();
     if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      prefetch_tmap(&tmdO);
-      mbar_expect_tx(kv_full, 2 * T);
-      for (int c = 0; c < kChunks; ++c) {
-        tma_load_3d(smem + L::kK + c * 16384, &tmK, 64 * c, n * kTile, bh, kv_full);
-        tma_load_3d(smem + L::kV + c * 16384, &tmV, 64 * c, n * kTile, bh, kv_full);
-      }
-      bool ok = true;
-      int issued = 0;
-      for (int mi = 0; mi < n_m; ++mi) {
-        const int m = m_begin + mi, st = mi & 1;
-        if (!(ok = wait(&q_empty[st], ((mi >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
-        mbar_expect_tx(&q_full[st], 2 * T + 1024);
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        prefetch_tmap(&tmdO);
+        mbar_expect_tx(kv_full, 2 * T);
         for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(smem + L::kQ + st * T + c * 16384, &tmQ, 64 * c, m * kTile, bh, &q_full[st]);
-          tma_load_3d(smem + L::kdO + st * T + c * 16384, &tmdO, 64 * c, m * kTile, bh, &q_full[st]);
+          tma_load_3d(smem + L::kK + c * 16384, &tmK, 64 * c, n * kTile, bh, kv_full);
+          tma_load_3d(smem + L::kV + c * 16384, &tmV, 64 * c, n * kTile, bh, kv_full);
         }
-        const size_t off = static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile;
-        bulk_load(smem + L::kLse + 512 * st, prm.nlse2 + off, 512, &q_full[st]);
-        bulk_load(smem + L::kDsum + 512 * st, prm.ndsum + off, 512, &q_full[st]);
-        ++issued;
+        bool ok = true;
+        int q_issued = 0, do_issued = 0;
+        for (int mi = 0; mi < n_m; ++mi) {
+          const int m = m_begin + mi, st = mi & 1;
+          // Q_m, -LSE2_m, -D_m into stage st (two stages)
+          if (!(ok = wait(&q_empty[st], ((mi >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
+          mbar_expect_tx(&q_full[st], T + 1024);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(smem + L::kQ + st * T + c * 16384, &tmQ, 64 * c, m * kTile, bh, &q_full[st]);
+          const size_t off = static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile;
+          bulk_load(smem + L::kLse + 512 * st, prm.nlse2 + off, 512, &q_full[st]);
+          bulk_load(smem + L::kDsum + 512 * st, prm.ndsum + off, 512, &q_full[st]);
+          ++q_issued;
+          // dO_m (one stage: free once dV_{m-1} has read it)
+          if (!(ok = wait(do_empty, (mi & 1) ^ 1, g, kSiteBwd | 14))) break;
+          mbar_expect_tx(do_full, T);
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(smem + L::kdO + c * 16384, &tmdO, 64 * c, m * kTile, bh, do_full);
+          ++do_issued;
+        }
+        if (!ok) {
+          drain_wait(kv_full, 0);
+          for (int i = q_issued - 2 > 0 ? q_issued - 2 : 0; i < q_issued; ++i)
+            drain_wait(&q_full[i & 1], (i >> 1) & 1);
+          if (do_issued > 0) drain_wait(do_full, (do_issued - 1) & 1);
+        }
       }
-      if (!ok) {
-        drain_wait(kv_full, 0);
-        for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i) drain_wait(&q_full[i & 1], (i >> 1) & 1);
-      }
-    }
     } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA
-    if (lane == 0) {
-      constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: both K-major
-      constexpr uint32_t idKM = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK: B MN-major
-      constexpr uint32_t idMM = idesc_bf16_f32(128, D, true, true);      // dQ: A and B MN-major
-      const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
-      const uint32_t sQ0 = smem_u32(smem + L::kQ), sdO0 = smem_u32(smem + L::kdO);
-      const uint32_t sdS = smem_u32(smem + L::kdS);
-      bool ok = wait(kv_full, 0, g, kSiteBwd | 2);
-      for (int mi = 0; ok && mi < n_m; ++mi) {
-        const int st = mi & 1;
-        const uint32_t ph = mi & 1;
-        const uint32_t sQ = sQ0 + st * T, sdO = sdO0 + st * T;
-        if (!(ok = wait(&q_full[st], (mi >> 1) & 1, g, kSiteBwd | 3))) break;
-        tc_fence_after();
-        // S^T = K Q^T
+      // ---------------------------------------------------------------- MMA
+      // Issue order per query tile m: dP_m, dV_m, S_{m+1}, dK_m, dQ_m -- S of the next tile is
+      // computed while the softmax warps turn dP_m into dS_m.
+      if (lane == 0) {
+        constexpr uint32_t idKK = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: both K-major
+        constexpr uint32_t idKM = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK: B MN-major
+        constexpr uint32_t idMM = idesc_bf16_f32(128, D, true, true);      // dQ: A and B MN-major
+        const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+        const uint32_t sQ0 = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO);
+        const uint32_t sdS = smem_u32(smem + L::kdS);
+        auto issue_s = [&](int st) {  // S^T = K Q^T
+          const uint32_t sQ = sQ0 + st * T;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + L::kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idKK, kk > 0);
-        }
-        tc_commit(s_full);
-        // dP^T = V dO^T (its columns hold dQ of the previous tile when aliased)
-        if (L::kAliasDQ && mi > 0) {
-          if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 4))) break;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + L::kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idKK,
+                   kk > 0);
+          }
+          tc_commit(s_full);
+        };
+        bool ok = wait(kv_full, 0, g, kSiteBwd | 2) && wait(&q_full[0], 0, g, kSiteBwd | 3);
+        if (ok) {
           tc_fence_after();
+          issue_s(0);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + L::kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024), idKK,
-                 kk > 0);
-        }
-        tc_commit(dp_full);
-        // dV += P^T dO
-        if (!(ok = wait(p_full, ph, g, kSiteBwd | 5))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + L::kColDV, tmem + L::kColS + 8 * kk, sdesc_sw128(sdO + kk * 2048, 16384, 1024), idKM,
-                 (mi > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q
-        if (!(ok = wait(ds_full, ph, g, kSiteBwd | 6))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
-                 idKM, (mi > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&q_empty[st]);  // Q_m, dO_m, -LSE2_m, -D_m no longer needed once these land
-        // dQ_m = dS K
-        if (!L::kAliasDQ && mi > 0) {
-          if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 7))) break;
+        for (int mi = 0; ok && mi < n_m; ++mi) {
+          const int st = mi & 1;
+          const uint32_t ph = mi & 1;
+          const uint32_t sQ = sQ0 + st * T;
+          // dP^T = V dO^T (its columns hold dQ of the previous tile when aliased)
+          if (!(ok = wait(do_full, ph, g, kSiteBwd | 15))) break;
+          if (L::kAliasDQ && mi > 0) {
+            if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 4))) break;
+          }
           tc_fence_after();
-        }
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ss(tmem + L::kColDQ, sdesc_sw128(sdS + kk * 2048, 16384, 1024),
-                 sdesc_sw128(sK + kk * 2048, 16384, 1024), idMM, kk > 0);
-        tc_commit(dq_full);
-        tc_commit(ds_empty);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + L::kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024), idKK,
+                   kk > 0);
+          }
+          tc_commit(dp_full);
+          // dV += P^T dO
+          if (!(ok = wait(p_full, ph, g, kSiteBwd | 5))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + L::kColDV, tmem + L::kColS + 8 * kk, sdesc_sw128(sdO + kk * 2048, 16384, 1024), idKM,
+                   (mi > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(do_empty);
+          // S^T of the next query tile (P_m in the S columns has been read by the dV MMA above)
+          if (mi + 1 < n_m) {
+            if (!(ok = wait(&q_full[st ^ 1], ((mi + 1) >> 1) & 1, g, kSiteBwd | 16))) break;
+            tc_fence_after();
+            issue_s(st ^ 1);
+          }
+          // dK += dS^T Q
+          if (!(ok = wait(ds_full, ph, g, kSiteBwd | 6))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
+                   idKM, (mi > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&q_empty[st]);  // Q_m, -LSE2_m, -D_m no longer needed once these land
+          // dQ_m = dS K
+          if (!L::kAliasDQ && mi > 0) {
+            if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 7))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ss(tmem + L::kColDQ, sdesc_sw128(sdS + kk * 2048, 16384, 1024),
+                   sdesc_sw128(sK + kk * 2048, 16384, 1024), idMM, kk > 0);
+          tc_commit(dq_full);
+          tc_commit(ds_empty);
+        }
+        if (ok) tc_commit(acc_full);
+        tc_commit(drain);
+        drain_wait(drain, 0);
       }
-      if (ok) tc_commit(acc_full);
-      tc_commit(drain);
-      drain_wait(drain, 0);
-    }
     }
   } else if (warp < 8) {
     regs_inc<kBwdRegsP>();
@@ -261,8 +288,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int ii = i + 2 * h;
-            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[cc][ii & 31]), __uint_as_float(sr[cc][(ii + 1) & 31])),
-                                        c2, h == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
+            const float2 x =
+                __ffma2_rn(make_float2(__uint_as_float(sr[cc][ii & 31]), __uint_as_float(sr[cc][(ii + 1) & 31])), c2,
+                           h == 0 ? make_float2(nl.x, nl.y) : make_float2(nl.z, nl.w));
             float2 pv;
             if (!edge && ((ii >> 1) & 7) < POLY16 / 2) {
               pv = exp2_poly2(x);
@@ -290,21 +318,27 @@ __global__ void __launch_bounds__(384, 1)
       if (mi > 0) {
         if (!(ok = wait_warp(ds_empty, ph ^ 1, g, kSiteBwd | 10))) break;
       }
+      uint32_t dp_[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t dp[32];
-        tmem_ld32(tdP + 32 * c, dp);
-        tmem_wait_ld();
-        reg_fence(dp);
+        if ((c & 1) == 0) {  // dP^T columns 64 at a time
+          tmem_ld32(tdP + 32 * c, dp_[0]);
+          tmem_ld32(tdP + 32 * c + 32, dp_[1]);
+          tmem_wait_ld();
+          reg_fence(dp_[0]);
+          reg_fence(dp_[1]);
+        }
+        uint32_t(&dpc)[32] = dp_[c & 1];
         uint32_t w[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const int i = 32 * c + 4 * e4;
           const float4 nd = nd4[i >> 2];
-          const float2 t0 = __fadd2_rn(make_float2(__uint_as_float(dp[4 * e4]), __uint_as_float(dp[4 * e4 + 1])),
-                                       make_float2(nd.x, nd.y));
-          const float2 t1 = __fadd2_rn(make_float2(__uint_as_float(dp[4 * e4 + 2]), __uint_as_float(dp[4 * e4 + 3])),
-                                       make_float2(nd.z, nd.w));
+          const float2 t0 = __fadd2_rn(
+              make_float2(__uint_as_float(dpc[4 * e4]), __uint_as_float(dpc[4 * e4 + 1])), make_float2(nd.x, nd.y));
+          const float2 t1 =
+              __fadd2_rn(make_float2(__uint_as_float(dpc[4 * e4 + 2]), __uint_as_float(dpc[4 * e4 + 3])),
+                         make_float2(nd.z, nd.w));
           const float2 d0 = __fmul2_rn(make_float2(p[i], p[i + 1]), t0);
           const float2 d1 = __fmul2_rn(make_float2(p[i + 2], p[i + 3]), t1);
           w[2 * e4] = pack_bf16x2(d0.x, d0.y);
@@ -353,31 +387,47 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else {
-    regs_dec<kBwdRegsDQ>();
-    // ----------------------------------------------------------- dQ drain
+    regs_inc<kBwdRegsDQ>();
+    // ---------------------------------------------------------- dQ drain
+    // dQ_m (fp32, in TMEM) leaves 32 columns at a time through a swizzled shared-memory staging
+    // buffer and a TMA reduce-add into the fp32 accumulator (two buffers, ping-pong).
     const int quarter = warp & 3;
     const int i = quarter * 32 + lane;  // query row within the tile
+    const bool leader = (warp == 8 && lane == 0);
     const uint32_t tdQ = tmem + L::kColDQ + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint8_t* stage0 = smem + L::kDQ;
+    if (leader) prefetch_tmap(&tmdQacc);
+    int flushed = 0;  // quarter tiles handed to TMA so far
     for (int mi = 0; mi < n_m; ++mi) {
       const int m = m_begin + mi;
       if (!wait_warp(dq_full, mi & 1, g, kSiteBwd | 12)) break;
       tc_fence_after();
-      float4* acc = reinterpret_cast<float4*>(
-          prm.dq_acc + (static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile + i) * D);
+      uint32_t a[D / 32][32];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tdQ + 32 * c, a);
-        tmem_wait_ld();
-        reg_fence(a);
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tdQ + 32 * c, a[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence(a[c]);
+      tc_fence_before();
+      mbar_arrive(dq_free);  // the dQ columns may be overwritten now
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c, ++flushed) {
+        uint8_t* buf = stage0 + (flushed & 1) * 16384;
+        if (leader) bulk_wait_read<1>();  // the reduce that last used this buffer has read it
+        named_barrier(1, 128);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
-          atomicAdd(acc + 8 * c + v, make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
-                                                 __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3])));
+          *reinterpret_cast<uint4*>(buf + i * 128 + (((v ^ i) & 7) << 4)) =
+              make_uint4(a[c][4 * v], a[c][4 * v + 1], a[c][4 * v + 2], a[c][4 * v + 3]);
+        fence_proxy_async();
+        named_barrier(1, 128);
+        if (leader) {
+          tma_reduce_add_3d(&tmdQacc, 32 * c, m * kTile, bh, buf);
+          bulk_commit();
+        }
       }
-      tc_fence_before();
-      mbar_arrive(dq_free);
     }
+    if (leader) bulk_wait<0>();
   }
 
   tc_fence_before();
