@@ -17,7 +17,8 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kPoly16 = 4;  // exponentials per 16 evaluated by the cubic when the polynomial path is on
+constexpr int kPoly16 = 4;     // exponentials per 16 evaluated by the cubic when the polynomial path is on
+constexpr int kBwdPoly16 = 0;  // backward: the SFU alone measured faster than any polynomial share
 
 __device__ int g_status;  // first device-side failure (wait site), 0 = none
 
@@ -29,7 +30,7 @@ struct DeviceState {
 DeviceState g_dev[kMaxDevices];
 
 float g_tau = fa::kRescaleTau;
-int g_poly = 1;
+int g_poly = 0;  // forward default: SFU only (measured faster on B200 than the 1/4 polynomial share)
 cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // one-shot [fwd|bwd][start|stop]
 
 // Records the pending start event of `which` (if any) on `st`; returns whether one was pending.
@@ -148,7 +149,7 @@ template <int D, bool C>
 int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
                const CUtensorMap& dq_acc, const fa::BwdParams& prm, cudaStream_t st) {
   using L = fa::BwdLayout<D>;
-  auto kern = fa::bwd_kernel<D, C, kPoly16>;
+  auto kern = fa::bwd_kernel<D, C, kBwdPoly16>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
   kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);

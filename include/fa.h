@@ -99,9 +99,9 @@ int fa_last_device_status(void* stream, int* detail);
 /*
  * Tuning of the forward softmax (process-wide; for A/B comparisons).
  * tau: rescale threshold in log2 units (0 <= tau <= 16; 0 = rescale whenever
- * the running maximum grows).  poly: 1 = evaluate a quarter of the
- * exponentials of interior tiles with the FMA-pipe cubic, 0 = all on the SFU.
- * Returns FA_ERR_INVALID_ARG for values out of range.
+ * the running maximum grows; default 8).  poly: 1 = evaluate a quarter of the
+ * exponentials of interior tiles with the FMA-pipe cubic, 0 = all on the SFU
+ * (default 0).  Returns FA_ERR_INVALID_ARG for values out of range.
  */
 int fa_set_softmax_options(float tau, int poly);
 

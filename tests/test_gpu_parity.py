@@ -21,7 +21,7 @@ def _device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     build.build()
-    api.fa_set_softmax_options(8.0, 1)
+    api.fa_set_softmax_options(8.0, 0)
     yield
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == (0, 0)
@@ -140,13 +140,13 @@ def test_several_tiles_and_heads_full(d, causal):
 @pytest.mark.parametrize("tau,poly", [(8.0, 1), (0.0, 0), (0.0, 1), (8.0, 0)])
 def test_rescale_and_exp_variants_agree(tau, poly):
     c = Case(1, 4, 2048, 128, False, seed_workload=3, stress=True)
-    api.fa_set_softmax_options(8.0, 1)
+    api.fa_set_softmax_options(8.0, 0)
     o_ref_gpu, lse_ref_gpu = c.fwd_gpu()
     try:
         api.fa_set_softmax_options(tau, poly)
         o, lse = c.fwd_gpu()
     finally:
-        api.fa_set_softmax_options(8.0, 1)
+        api.fa_set_softmax_options(8.0, 0)
     check_fwd(c, o, lse, all_heads(c), 128, f"variant tau={tau} poly={poly}")
     assert float((o.float() - o_ref_gpu.float()).abs().max()) <= TOL_O
     assert float((lse - lse_ref_gpu).abs().max()) <= TOL_LSE
