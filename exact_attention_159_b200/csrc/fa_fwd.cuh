@@ -5,14 +5,17 @@
 // works for one tile, the softmax warps work on the other).  Warp roles
 // ("The Technical Edge": warp specialisation into load / MMA / softmax /
 // output stages):
-//   warp 0      TMA producer: Q tiles once, then a ring of K/V tiles
-//   warp 1      MMA issuer (one thread) and TMEM owner
-//   warps 2, 3  idle (they complete the first warpgroup)
-//   warps 4..7  softmax + correction + epilogue for query tile 0
-//   warps 8..11 the same for query tile 1
-// Registers are re-split per warpgroup with setmaxnreg (56 / 224 / 224 of
-// the 168 x 384 launched), so the softmax rows (128 fp32 scores each) stay in
-// registers.  The softmax arithmetic uses packed fp32x2 FMA/add.
+//   warp 0        TMA producer: Q tiles once, then a ring of K/V tiles
+//   warp 1        MMA issuer (one thread) and TMEM owner
+//   warps 2, 3    idle (they complete the first warpgroup)
+//   warps 4..11   softmax + correction + epilogue for query tile 0
+//   warps 12..19  the same for query tile 1
+// Every score row is split between two threads (two warps on the same TMEM
+// lane quarter): each takes 64 of the 128 key columns, and the pair agrees on
+// the row maximum through shared memory and a 64-thread named barrier.  Four
+// softmax warps per SM sub-partition hide the SFU and TMEM latencies.
+// Registers are re-split per warpgroup with setmaxnreg (56 / 104 of the
+// 96 x 640 launched).  The softmax arithmetic uses packed fp32x2 FMA/add.
 // Tensor memory (512 columns x 128 lanes x 32 bit, "TMEM (256 KB per SM)"):
 //   S_t = Q_t K^T  fp32, 128 columns at 128*t; P_t (bf16, packed two per
 //   column) is written back over the first 64 columns of S_t and read from
@@ -61,8 +64,9 @@ struct FwdLayout {
   // q, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
   static constexpr int kNumBars = 1 + 3 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 16;  // the dynamic shared memory base is 1024-byte aligned
-  static constexpr int kThreads = 384;
+  static constexpr int kXchg = kMisc + 16;     // [tile][half][row] fp32 row-max / row-sum exchange
+  static constexpr int kBytes = kXchg + 2 * 2 * 128 * 4;  // the dynamic shared memory base is 1024-byte aligned
+  static constexpr int kThreads = 640;
 };
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight async work).
@@ -73,12 +77,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Register split (setmaxnreg): 128 * (56 + 224 + 224) = 384 * 168, the launch's total.  Each
+// Register split (setmaxnreg): 128 * 56 + 512 * 104 <= 640 * 96, the launch's total.  Each
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
-constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 224;
+constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 104;
 
 template <int D, bool CAUSAL, int POLY16>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
   using L = FwdLayout<D>;
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 256);
       mbar_init(&o_full[t], 1);
     }
     mbar_init(drain, 1);
@@ -230,73 +234,63 @@ __global__ void __launch_bounds__(384, 1)
   } else {
     regs_inc<kFwdRegsSoftmax>();
     // ------------------------------------------- softmax / correction / epilogue
-    const int t = (warp >> 2) - 1;
-    const int quarter = warp & 3;  // TMEM lanes this warp may touch: 32*quarter .. +31
+    const int t = (warp - 4) >> 3;        // query tile
+    const int h = ((warp - 4) >> 2) & 1;  // which 64 key columns of the row (and D/2 columns of O)
+    const int quarter = warp & 3;         // TMEM lanes this warp may touch: 32*quarter .. +31
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + 128 * t + lane_off;
-    const uint32_t tO = tmem + 256 + D * t + lane_off;
+    const uint32_t tO = tmem + 256 + D * t + (D / 2) * h + lane_off;
+    float* xchg = reinterpret_cast<float*>(smem + L::kXchg) + t * 256;  // [half][row]
+    const int bar_id = 1 + 4 * t + quarter;                            // the two warps sharing these rows
     const int qt = 2 * pair + t;
     const int row = qt * kTile + r;  // query row within the head
     const float sl2 = prm.scale_log2;
-    float m_ref = -INFINITY, l = 0.0f;
+    float m_ref = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
     bool ok = true;
     for (int j = 0; j < nkv[t]; ++j) {
       if (!(ok = wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7))) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
+      uint32_t sr[2][32];
+      tmem_ld32(tS + 64 * h, sr[0]);
+      tmem_ld32(tS + 64 * h + 32, sr[1]);
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-      // scores stay in the registers tcgen05.ld wrote (S(c) reads column c as fp32)
+      reg_fence(sr[0]);
+      reg_fence(sr[1]);
+      // scores stay in the registers tcgen05.ld wrote (S(c) reads local column c as fp32)
 #define S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
       const bool edge = (CAUSAL && j == qt) || ((j + 1) * kTile > prm.N);
       if (edge) {
-        const int key0 = j * kTile;
+        const int key0 = j * kTile + 64 * h;
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) {
+        for (int c = 0; c < 64; ++c) {
           const int key = key0 + c;
           if (key >= prm.N || (CAUSAL && key > row)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
       }
-      // row maximum: four independent chains of 3-input max
-      float mx[4] = {S(0), S(32), S(64), S(96)};
+      // row maximum: two chains of 3-input max over this half, then the partner's half
+      float mx[2] = {S(0), S(32)};
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 2; ++q)
 #pragma unroll
         for (int c = 32 * q + 1; c < 32 * q + 31; c += 2) mx[q] = fmax3(mx[q], S(c), S(c + 1));
 #pragma unroll
-      for (int q = 0; q < 4; ++q) mx[q] = fmaxf(mx[q], S(32 * q + 31));
-      const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2);
-      const bool need = m_new > m_ref + prm.tau;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // correction: O_t *= 2^(m_ref - m_new) once the previous P.V has landed
-        if (!(ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8))) break;
-        tc_fence_after();
-        const float alpha = need ? exp2_sfu(m_ref - m_new) : 1.0f;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
-          reg_fence(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
-        tmem_wait_st();
-      }
+      for (int q = 0; q < 2; ++q) mx[q] = fmaxf(mx[q], S(32 * q + 31));
+      const float mine = fmaxf(mx[0], mx[1]);
+      xchg[128 * h + r] = mine;
+      named_barrier(bar_id, 64);
+      const float m_new = fmaxf(m_ref, fmaxf(mine, xchg[128 * (h ^ 1) + r]) * sl2);
+      const bool need = m_new > m_ref + prm.tau;  // identical in both threads of the row
+      const float alpha = need ? exp2_sfu(m_ref - m_new) : 1.0f;
       if (need) {
-        l *= exp2_sfu(m_ref - m_new);
+        l *= alpha;
         m_ref = m_new;
       }
       // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 columns at a time)
       const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
       float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -315,11 +309,27 @@ __global__ void __launch_bounds__(384, 1)
             ls0 = __fadd2_rn(ls0, p);
           pk[e] = pack_bf16x2(p.x, p.y);
         }
-        tmem_st16(tS + 16 * cc, pk);
+        tmem_st16(tS + 32 * h + 16 * cc, pk);
       }
 #undef S
       const float2 ls = __fadd2_rn(ls0, ls1);
       l += ls.x + ls.y;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // correction: this thread's half of O_t *= alpha once the previous P.V has landed (before
+        // p_full lets the next P.V accumulate into it)
+        if (!(ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
@@ -327,11 +337,15 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && nkv[t] > 0) ok = wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
     if (ok && nkv[t] > 0) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      // full row sum from the two halves
+      xchg[128 * h + r] = l;
+      named_barrier(bar_id, 64);
+      const float l_row = l + xchg[128 * (h ^ 1) + r];
+      const float inv_l = 1.0f / l_row;
       const bool store = row < prm.N;
-      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D;
+      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D + (D / 2) * h;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_wait_ld();
@@ -346,7 +360,8 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (store) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = (m_ref + log2f(l)) * 0.69314718055994531f;
+      if (store && h == 0)
+        prm.LSE[static_cast<size_t>(bh) * prm.N + row] = (m_ref + log2f(l_row)) * 0.69314718055994531f;
     }
   }
 
