@@ -90,8 +90,8 @@ __global__ void __launch_bounds__(384, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % prm.BH;
-  const int n = blockIdx.x / prm.BH;          // key tile; n = 0 has the most causal work
+  int bh, n;  // key tile n = 0 (the most causal work) first, a few heads at a time
+  cta_order(blockIdx.x, prm.BH, prm.n_tiles, bh, n);
   const int m_begin = CAUSAL ? n : 0;
   const int n_m = prm.n_tiles - m_begin;      // >= 1
 

@@ -108,8 +108,9 @@ __global__ void __launch_bounds__(640, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % prm.BH;
-  const int pair = prm.n_pairs - 1 - blockIdx.x / prm.BH;  // heaviest causal work first
+  int bh, unit;  // heaviest causal work (the last query tiles) first, a few heads at a time
+  cta_order(blockIdx.x, prm.BH, prm.n_pairs, bh, unit);
+  const int pair = prm.n_pairs - 1 - unit;
   const int n_tiles = (prm.N + kTile - 1) / kTile;
   int nkv[2];
 #pragma unroll

@@ -238,6 +238,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// CTA order for causal work lists: heads are taken in groups of kHeadGroup (so the CTAs running
+// at one time share a few heads' streamed tiles in L2), heaviest unit first inside a group with the
+// head as the fast index.  Returns the head and the unit index (0 = heaviest).
+constexpr int kHeadGroup = 2;
+__device__ __forceinline__ void cta_order(int cta, int n_heads, int n_units, int& head, int& unit) {
+  const int g = cta / (kHeadGroup * n_units);
+  const int heads_here = min(kHeadGroup, n_heads - g * kHeadGroup);
+  const int r = cta - g * kHeadGroup * n_units;
+  unit = r / heads_here;
+  head = g * kHeadGroup + r % heads_here;
+}
+
 // ------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (tiles written by TMA with
 // CU_TENSOR_MAP_SWIZZLE_128B, or by threads with the same XOR pattern, from a
