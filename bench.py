@@ -50,6 +50,35 @@ def peaks():
         return dict(burst=1590.0, sustained=1400.0, hbm=6650.0, source="fallback")
 
 
+KERNEL_SOURCES = ("fa_fwd.cuh", "fa_bwd.cuh", "sm100.cuh", "exp2_poly.cuh")
+
+
+def kernel_source_hash():
+    """SHA-256 over the kernel sources; a stored ncu traffic figure is only valid for the same hash."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "exact_attention_159_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def stored_traffic(kernel):
+    """DRAM bytes per launch of `kernel` ("fwd" or "bwd") from the committed ncu summary of the bench
+    workload, or None when the summary is missing or was taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic_long_context_causal_B1_H16_N32768_d128.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    import re
+    src = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    val = re.search(rf"{kernel}_traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not src or not val or src.group(1) != kernel_source_hash():
+        return None
+    return int(val.group(1))
+
+
 def config_dict(n_gpus):
     w = WORKLOAD
     return {"workload": f"{w['name']}: B={w['B']} H={w['H']} N={w['N']} d={w['d']}",
@@ -114,6 +143,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------- multi-rank
+def rank_seed(workload_seed, rank):
+    """Seed of a rank's inputs: every rank draws its own heads (weak scaling)."""
+    return workload_seed + 100 * rank
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max over ranks of per-rank timings (a collective only when world > 1)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tflops(flops_per_rank, world, ms_per_step):
+    """Whole-job throughput: the work of every rank divided by the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args):
     import numpy as np
@@ -135,7 +185,7 @@ def run_gpu(args):
     B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
     scale = 1.0 / math.sqrt(d)
     # each rank draws its own heads (weak scaling): shift the seed by rank
-    bits = I.attention_inputs(w["seed_workload"] + 100 * rank, B, H, N, d, with_do=True)
+    bits = I.attention_inputs(rank_seed(w["seed_workload"], rank), B, H, N, d, with_do=True)
     host = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory() for k, v in bits.items()}
     dev = {k: v.cuda() for k, v in host.items()}
     o = torch.empty_like(dev["q"])
@@ -211,14 +261,10 @@ def run_gpu(args):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    vals = torch.tensor([ms, e2e_ms, max(fwd_ms), max(bwd_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, e2e_ms = float(vals[0]), float(vals[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, "cuda")
     f_fwd, f_bwd = flops(B, H, N, d, causal)
-    step_flops = (f_fwd + f_bwd) * world
     ms_step = ms / args.steps
-    value = step_flops / (ms_step * 1e-3) / 1e12
+    value = job_tflops(f_fwd + f_bwd, world, ms_step)
     pk = peaks()
     fwd_avg = statistics.mean(fwd_ms)
     bwd_avg = statistics.mean(bwd_ms)
@@ -242,8 +288,9 @@ def run_gpu(args):
         "roofline": {"bound": "tensor", "kernel": f"{dominant} attention kernel", "achieved": round(ach, 2),
                      "peak": pk["sustained"], "unit": "TFLOP/s", "frac": round(ach / pk["sustained"], 4),
                      "peak_kind": f"{pk['source']} sustained bf16 (kernel timed inside a multi-second loop)",
-                     "traffic": None},
-        "e2e": {"value": round(step_flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                     "traffic": stored_traffic(dominant),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
+        "e2e": {"value": round(job_tflops(f_fwd + f_bwd, world, e2e_ms), 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
                 "ms_per_step": round(e2e_ms, 3)},
         "gpu_launches": 4 * args.steps,
@@ -374,8 +421,12 @@ def main():
     ap.add_argument("--profile", choices=["fwd", "bwd"], help="plain calls on --shape for ncu captures")
     ap.add_argument("--shape", default="1,16,16384,128", help="B,H,N,d for --profile")
     ap.add_argument("--causal", type=int, default=1, help="causal flag for --profile")
+    ap.add_argument("--source-hash", action="store_true", help="print the kernel source hash and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.source_hash:
+        print(kernel_source_hash())
+        return
     if args.profile:
         run_profile(args)
     elif args.impl == "reference":

@@ -31,6 +31,7 @@ SIGNATURES = {
     "fa_exp2_eval": (_I, [_P, _P, ctypes.c_int64, _I, _P]),
     "fa_profile_next": (_I, [_I, _P, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
+    "fa_selftest_wait_timeout": (_I, [_P]),
     "fa_version": (_I, []),
 }
 

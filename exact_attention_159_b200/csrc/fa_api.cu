@@ -170,6 +170,22 @@ WsLayout ws_layout(long long BH, int N, int d) {
   return w;
 }
 
+// One CTA waits on a barrier that never completes: exercises the bounded-wait failure path.
+__global__ void selftest_wait_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(&bar, 1);
+    abort_flag = 0;
+    fa::fence_mbar_init();
+  }
+  __syncthreads();
+  const fa::Guard g{&abort_flag, status};
+  fa::wait_warp(&bar, 0, g, 0xF01);  // nobody arrives: gives up after the wait limit
+  __syncthreads();
+  if (threadIdx.x == 0) fa::mbar_arrive(&bar);  // complete the phase so the barrier is left idle
+}
+
 __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int mode) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
@@ -414,6 +430,14 @@ int fa_profile_next(int which, void* start_event, void* stop_event) {
   g_prof[which][0] = static_cast<cudaEvent_t>(start_event);
   g_prof[which][1] = static_cast<cudaEvent_t>(stop_event);
   return FA_OK;
+}
+
+int fa_selftest_wait_timeout(void* stream) {
+  int rc = FA_OK;
+  int* status = device_status(&rc);
+  if (!status) return rc;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream) {

@@ -124,6 +124,17 @@ int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
  */
 int fa_profile_next(int which, void* start_event, void* stop_event);
 
+/*
+ * Failure-path self test: launches one small kernel on `stream` whose only
+ * pipeline wait is on a barrier that nothing ever arrives at.  The bounded
+ * wait used by every kernel of the library gives up after its limit (2 s),
+ * records its site in the device status word and the kernel returns; no
+ * fault, trap or hang is involved.  A following fa_last_device_status(stream)
+ * must then report FA_ERR_TIMEOUT with detail 0xF01.  Returns the launch
+ * status.
+ */
+int fa_selftest_wait_timeout(void* stream);
+
 /* Size of the fixed device scratch array behind fa_bwd_noalloc (64 MiB). */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 
