@@ -104,8 +104,12 @@ def fa_last_device_status(stream=None) -> tuple[int, int]:
     return int(rc), int(detail.value)
 
 
-def fa_set_softmax_options(tau: float = 8.0, poly: int = 1) -> None:
+def fa_set_softmax_options(tau: float = 8.0, poly: int = 0) -> None:
     check(_lib.lib().fa_set_softmax_options(float(tau), int(poly)), "fa_set_softmax_options")
+
+
+def fa_set_forward_variant(cluster_pair: int = 0) -> None:
+    check(_lib.lib().fa_set_forward_variant(int(cluster_pair)), "fa_set_forward_variant")
 
 
 def fa_exp2_eval(x: torch.Tensor, mode: int = 0, stream=None) -> torch.Tensor:

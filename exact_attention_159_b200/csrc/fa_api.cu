@@ -13,6 +13,7 @@
 #include "exp2_poly.cuh"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd2.cuh"
 
 namespace {
 
@@ -31,6 +32,7 @@ DeviceState g_dev[kMaxDevices];
 
 float g_tau = fa::kRescaleTau;
 int g_poly = 0;  // forward default: SFU only (measured faster on B200 than the 1/4 polynomial share)
+int g_fwd_pair = 0;  // 1: forward at d = 128 on cluster pairs (cta_group::2 UMMA)
 cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // one-shot [fwd|bwd][start|stop]
 
 // Records the pending start event of `which` (if any) on `st`; returns whether one was pending.
@@ -82,13 +84,13 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// 3-D map over a contiguous [BH, N, d] bf16 tensor: box 64 (d) x 128 (rows) x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d) {
+// 3-D map over a contiguous [BH, N, d] bf16 tensor: box 64 (d) x `rows` x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -142,6 +144,16 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_pairs);
   kern<<<grid, L::kThreads, L::kBytes, st>>>(q, k, v, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool C, int P>
+int launch_fwd2(const CUtensorMap& q, const CUtensorMap& k64, const CUtensorMap& v, const fa::Fwd2Params& prm,
+                cudaStream_t st) {
+  auto kern = fa::fwd2_kernel<C, P>;
+  if (set_smem(kern, fa::Fwd2Layout::kBytes) != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = 2u * static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_quads);
+  kern<<<grid, fa::Fwd2Layout::kThreads, fa::Fwd2Layout::kBytes, st>>>(q, k64, v, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -254,6 +266,26 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   prm.status = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool poly = g_poly != 0;
+  if (d == 128 && g_fwd_pair) {
+    CUtensorMap mk64;
+    if (!make_map(&mk64, K, BH, N, d, 64)) return FA_ERR_CUDA;
+    fa::Fwd2Params p2;
+    p2.O = prm.O;
+    p2.LSE = prm.LSE;
+    p2.N = N;
+    p2.BH = BH;
+    p2.n_quads = (tiles + 3) / 4;
+    p2.scale_log2 = prm.scale_log2;
+    p2.tau = prm.tau;
+    p2.status = prm.status;
+    const bool prof2 = prof_begin(0, st);
+    if (causal)
+      rc = poly ? launch_fwd2<true, kPoly16>(mq, mk64, mv, p2, st) : launch_fwd2<true, 0>(mq, mk64, mv, p2, st);
+    else
+      rc = poly ? launch_fwd2<false, kPoly16>(mq, mk64, mv, p2, st) : launch_fwd2<false, 0>(mq, mk64, mv, p2, st);
+    if (prof2) prof_end(0, st);
+    return rc;
+  }
   const bool prof = prof_begin(0, st);
   if (d == 128) {
     if (causal)
@@ -422,6 +454,12 @@ int fa_last_device_status(void* stream, int* detail) {
     if (detail) *detail = v;
     return FA_ERR_TIMEOUT;
   }
+  return FA_OK;
+}
+
+int fa_set_forward_variant(int cluster_pair) {
+  if (cluster_pair != 0 && cluster_pair != 1) return FA_ERR_INVALID_ARG;
+  g_fwd_pair = cluster_pair;
   return FA_OK;
 }
 

@@ -397,10 +397,14 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tdQ = tmem + L::kColDQ + (static_cast<uint32_t>(quarter * 32) << 16);
     uint8_t* stage0 = smem + L::kDQ;
     if (leader) prefetch_tmap(&tmdQacc);
+    // The four drain warps pass the same hardware barriers (id 1) in the same order; the only
+    // wait that can fail (dq_full) is followed by a joint decision, so they leave together.
     int flushed = 0;  // quarter tiles handed to TMA so far
+    bool ok = true;
     for (int mi = 0; mi < n_m; ++mi) {
       const int m = m_begin + mi;
-      if (!wait_warp(dq_full, mi & 1, g, kSiteBwd | 12)) break;
+      const bool okl = ok && wait_warp(dq_full, mi & 1, g, kSiteBwd | 12);
+      if (!(ok = group_and(1, 128, okl))) break;
       tc_fence_after();
       uint32_t a[D / 32][32];
 #pragma unroll

@@ -250,7 +250,10 @@ __global__ void __launch_bounds__(640, 1)
     float m_ref = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
     bool ok = true;
     for (int j = 0; j < nkv[t]; ++j) {
-      if (!(ok = wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7))) break;
+      // every exit decision is taken jointly by the two warps of a row (group_and), so neither is
+      // ever left waiting at a barrier the other skipped; after a failed wait the block below
+      // only reads stale TMEM columns of this CTA's own allocation before the joint exit
+      const bool okl = ok && wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7);
       tc_fence_after();
       uint32_t sr[2][32];
       tmem_ld32(tS + 64 * h, sr[0]);
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(640, 1)
       for (int q = 0; q < 2; ++q) mx[q] = fmaxf(mx[q], S(32 * q + 31));
       const float mine = fmaxf(mx[0], mx[1]);
       xchg[128 * h + r] = mine;
-      named_barrier(bar_id, 64);
+      if (!(ok = group_and(bar_id, 64, okl))) break;
       const float m_new = fmaxf(m_ref, fmaxf(mine, xchg[128 * (h ^ 1) + r]) * sl2);
       const bool need = m_new > m_ref + prm.tau;  // identical in both threads of the row
       const float alpha = need ? exp2_sfu(m_ref - m_new) : 1.0f;
@@ -318,8 +321,8 @@ __global__ void __launch_bounds__(640, 1)
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // correction: this thread's half of O_t *= alpha once the previous P.V has landed (before
         // p_full lets the next P.V accumulate into it)
-        if (!(ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8))) break;
-        tc_fence_after();
+        ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8);
+        tc_fence_after();  // a failed wait is carried to the next joint decision
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t o[32];
@@ -333,14 +336,18 @@ __global__ void __launch_bounds__(640, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      if (ok) mbar_arrive(&p_full[t]);
     }
-    if (ok && nkv[t] > 0) ok = wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
+    if (nkv[t] > 0) {
+      // full row sum from the two halves (joint decision, as in the loop)
+      const bool okl = ok && wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
+      if (okl) {
+        tc_fence_after();
+        xchg[128 * h + r] = l;
+      }
+      ok = group_and(bar_id, 64, okl);
+    }
     if (ok && nkv[t] > 0) {
-      tc_fence_after();
-      // full row sum from the two halves
-      xchg[128 * h + r] = l;
-      named_barrier(bar_id, 64);
       const float l_row = l + xchg[128 * (h ^ 1) + r];
       const float inv_l = 1.0f / l_row;
       const bool store = row < prm.N;

@@ -106,6 +106,16 @@ int fa_last_device_status(void* stream, int* detail);
 int fa_set_softmax_options(float tau, int poly);
 
 /*
+ * Forward kernel selection (process-wide; for A/B comparisons).  0 (default):
+ * the single-CTA kernel.  1: at d = 128 the forward runs on cluster pairs of
+ * SMs, every MMA a 2-SM (cta_group::2) UMMA of M = 256 with K and V split
+ * between the pair (same results, currently slower).  d = 64 always uses the
+ * single-CTA kernel.
+ * Returns FA_ERR_INVALID_ARG for other values.
+ */
+int fa_set_forward_variant(int cluster_pair);
+
+/*
  * Elementwise y = 2^x on the device for testing the exponential the kernels
  * use: mode 0 = the cubic-polynomial software exp2, mode 1 = the SFU
  * (ex2.approx), mode 2 = the cubic with packed fp32x2 arithmetic on element

@@ -181,3 +181,32 @@ def test_unsupported_head_dim_launches_nothing():
     with pytest.raises(_lib.FAError) as e:
         api.fa_fwd(q, q.clone(), q.clone())
     assert e.value.code == _lib.FA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------ forward kernel variants
+VARIANT_SHAPES = [(1, 2, 200, True), (2, 3, 640, False), (1, 2, 640, True), (1, 4, 1000, True), (1, 2, 1536, False),
+                  (2, 2, 2048, True)]
+
+
+@pytest.mark.parametrize("variant", [0, 1], ids=["single-cta", "cluster-pair"])
+@pytest.mark.parametrize("B,H,N,causal", VARIANT_SHAPES, ids=[f"B{b}H{h}N{n}{'c' if c else 'f'}" for b, h, n, c in VARIANT_SHAPES])
+def test_forward_variants_full(variant, B, H, N, causal):
+    c = Case(B, H, N, 128, causal, seed_workload=14)
+    api.fa_set_forward_variant(variant)
+    try:
+        o, lse = c.fwd_gpu()
+    finally:
+        api.fa_set_forward_variant(0)
+    check_fwd(c, o, lse, all_heads(c), None if N <= 1000 else 160, f"variant {variant} B{B} H{H} N{N} c{int(causal)}")
+
+
+def test_forward_variants_agree_at_full_size():
+    c = Case(1, 16, 32768, 128, True, seed_workload=4)
+    o0, l0 = c.fwd_gpu()
+    api.fa_set_forward_variant(1)
+    try:
+        o1, l1 = c.fwd_gpu()
+    finally:
+        api.fa_set_forward_variant(0)
+    assert float((o0.float() - o1.float()).abs().max()) <= 1e-2
+    assert float((l0 - l1).abs().max()) <= 1e-3
