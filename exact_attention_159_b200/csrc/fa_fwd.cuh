@@ -61,8 +61,8 @@ struct FwdLayout {
   static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
-  // q, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
-  static constexpr int kNumBars = 1 + 3 * kStages + 7;
+  // q, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kXchg = kMisc + 16;     // [tile][half][row] fp32 row-max / row-sum exchange
   static constexpr int kBytes = kXchg + 2 * 2 * 128 * 4;  // the dynamic shared memory base is 1024-byte aligned
@@ -99,8 +99,9 @@ __global__ void __launch_bounds__(640, 1)
   uint64_t* bar_q = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + S;
-  uint64_t* kv_empty = v_full + S;
-  uint64_t* s_full = kv_empty + S;
+  uint64_t* k_empty = v_full + S;  // K and V stages are released separately: K(j) is done
+  uint64_t* v_empty = k_empty + S;  // once both S(t, j) are, about an iteration before V(j)
+  uint64_t* s_full = v_empty + S;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = p_full + 2;
   uint64_t* drain = o_full + 2;
@@ -125,7 +126,8 @@ __global__ void __launch_bounds__(640, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -158,26 +160,27 @@ __global__ void __launch_bounds__(640, 1)
         if (nkv[t] > 0)
           for (int c = 0; c < kChunks; ++c)
             tma_load_3d(smem + L::kQ + t * T + c * 16384, &tmQ, 64 * c, (2 * pair + t) * kTile, bh, bar_q);
-      int issued = 0;
+      // K(j) then V(j): the order in which their stages are released
+      int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv_max; ++j) {
         const int s = j % S;
         const uint32_t ph = (j / S) & 1;
-        if (!(ok = wait(&kv_empty[s], ph ^ 1, g, kSiteFwd | 1))) break;
+        if (!(ok = wait(&k_empty[s], ph ^ 1, g, kSiteFwd | 1))) break;
         mbar_expect_tx(&k_full[s], T);
         for (int c = 0; c < kChunks; ++c)
           tma_load_3d(smem + L::kK + s * T + c * 16384, &tmK, 64 * c, j * kTile, bh, &k_full[s]);
+        ++k_issued;
+        if (!(ok = wait(&v_empty[s], ph ^ 1, g, kSiteFwd | 12))) break;
         mbar_expect_tx(&v_full[s], T);
         for (int c = 0; c < kChunks; ++c)
           tma_load_3d(smem + L::kV + s * T + c * 16384, &tmV, 64 * c, j * kTile, bh, &v_full[s]);
-        ++issued;
+        ++v_issued;
       }
       if (!ok) {  // let copies already in flight land before the CTA exits
         drain_wait(bar_q, 0);
-        for (int i = issued - S > 0 ? issued - S : 0; i < issued; ++i) {
-          drain_wait(&k_full[i % S], (i / S) & 1);
-          drain_wait(&v_full[i % S], (i / S) & 1);
-        }
+        for (int i = k_issued - S > 0 ? k_issued - S : 0; i < k_issued; ++i) drain_wait(&k_full[i % S], (i / S) & 1);
+        for (int i = v_issued - S > 0 ? v_issued - S : 0; i < v_issued; ++i) drain_wait(&v_full[i % S], (i / S) & 1);
       }
     }
     } else if (warp == 1) {
@@ -208,6 +211,7 @@ __global__ void __launch_bounds__(640, 1)
             issue_s(t, 0);
             tc_commit(&s_full[t]);
           }
+        tc_commit(&k_empty[0]);  // K(0) is free once both S(t, 0) are done
       }
       for (int j = 0; ok && j < nkv_max; ++j) {
         const int s = j % S;
@@ -226,7 +230,10 @@ __global__ void __launch_bounds__(640, 1)
             tc_commit(&s_full[t]);
           }
         }
-        if (ok) tc_commit(&kv_empty[s]);
+        if (ok) {
+          tc_commit(&v_empty[s]);                                 // V(j): both P.V issued
+          if (j + 1 < nkv_max) tc_commit(&k_empty[(j + 1) % S]);  // K(j+1): both S(t, j+1) issued
+        }
       }
       tc_commit(drain);
       drain_wait(drain, 0);

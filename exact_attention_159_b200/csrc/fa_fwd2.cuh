@@ -310,7 +310,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (ok && lane == 0) mbar_arrive_cluster(p_full0);
+      // P and the corrected O are tensor memory, complete after tcgen05.wait::st: a relaxed arrival
+      if (ok && lane == 0) mbar_arrive_cluster_relaxed(p_full0);
     }
     if (nkv[t] > 0) {
       // full row sum from the two halves (joint decision, as in the loop)

@@ -309,6 +309,13 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Relaxed arrival on a barrier of a CTA of this cluster: no release of this thread's generic
+// memory operations, so it costs tens of cycles where the release form costs over a thousand.
+// Sufficient where the only data handed over is tensor memory that this thread has already
+// waited for (tcgen05.wait::st, then tcgen05.fence::before_thread_sync).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 // TMA tile load into this CTA's shared memory whose completion is counted on `bar` (a
 // shared::cluster address, here the leader CTA's barrier) -- the pair form used by 2-SM UMMA.
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
