@@ -249,7 +249,97 @@ def pin_row_subsets(lib):
         _close(dvs, dv[rows[::-1]], 0.0, "row subset dV")
 
 
+def _torch_masked(q, k, v, do, scale, causal, rows):
+    """torch fp64 attention with an explicit boolean mask (the last query aligned with the last
+    key) over the query ``rows`` that see at least one key, with autograd gradients."""
+    import torch
+    nq, nk = q.shape[0], k.shape[0]
+    i = np.asarray(rows)[:, None]
+    j = np.arange(nk)[None, :]
+    mask = (j <= i + (nk - nq)) if causal else np.ones((len(rows), nk), bool)
+    t = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q[rows], k, v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(t[0][None], t[1][None], t[2][None],
+                                                           attn_mask=torch.tensor(mask)[None], scale=scale)[0]
+    ref.backward(torch.tensor(do[rows]))
+    s = np.where(mask, scale * (q[rows] @ k.T), -np.inf)
+    lse = torch.logsumexp(torch.tensor(s), dim=1).numpy()
+    return ref.detach().numpy(), lse, t[0].grad.numpy(), t[1].grad.numpy(), t[2].grad.numpy()
+
+
+def pin_torch_rectangular(lib):
+    """nq != nk, causal aligned bottom-right: torch fp64 attention with an explicit mask + autograd
+    over the rows that see a key; the rows that see none are O = 0, LSE = -inf, dQ = 0 and add
+    nothing to dK, dV (so torch over the visible rows alone gives the same dK, dV)."""
+    for (nq, nk, d, causal, seed) in ((5, 11, 4, True, 31), (11, 5, 4, True, 32), (7, 13, 6, False, 33),
+                                      (1, 9, 3, True, 34), (16, 40, 8, True, 35), (40, 16, 8, True, 36)):
+        r = _rng(seed)
+        q, do = r.standard_normal((nq, d)), r.standard_normal((nq, d))
+        k, v = r.standard_normal((nk, d)), r.standard_normal((nk, d))
+        scale = 0.7 / math.sqrt(d)
+        seen = np.arange(nq) + (nk - nq) >= 0 if causal else np.ones(nq, bool)
+        rows = np.nonzero(seen)[0]
+        o_t, lse_t, dq_t, dk_t, dv_t = _torch_masked(q, k, v, do, scale, causal, rows)
+        o, lse = O.fwd(q, k, v, scale, causal, nthreads=3, lib=lib)
+        _close(o[rows], o_t, 1e-12, f"rect O {nq}x{nk}")
+        _close(lse[rows], lse_t, 1e-12, f"rect LSE {nq}x{nk}")
+        dq, dk, dv, lse2, _ = O.bwd(q, k, v, do, scale, causal, nthreads=2, lib=lib)
+        _close(dq[rows], dq_t, 1e-11, f"rect dQ {nq}x{nk}")
+        _close(dk, dk_t, 1e-11, f"rect dK {nq}x{nk}")
+        _close(dv, dv_t, 1e-11, f"rect dV {nq}x{nk}")
+        blind = np.nonzero(~seen)[0]
+        if blind.size:
+            _close(o[blind], np.zeros((blind.size, d)), 0.0, "masked rows O = 0")
+            _close(dq[blind], np.zeros((blind.size, d)), 0.0, "masked rows dQ = 0")
+            assert np.all(np.isneginf(lse[blind])) and np.all(np.isneginf(lse2[blind])), "masked rows LSE = -inf"
+
+
+def pin_cache_suffix(lib):
+    """Causal nq < nk (new queries over a cache of earlier keys) equals the last nq rows of the
+    square causal problem whose last nq queries are those; with the earlier rows' dO = 0 the
+    square problem's dK, dV equal the rectangular ones."""
+    nq, nk, d = 6, 15, 5
+    r = _rng(37)
+    qfull, dofull = r.standard_normal((nk, d)), r.standard_normal((nk, d))
+    dofull[: nk - nq] = 0.0
+    k, v = r.standard_normal((nk, d)), r.standard_normal((nk, d))
+    q, do = qfull[nk - nq:], dofull[nk - nq:]
+    o, lse = O.fwd(q, k, v, 0.6, True, nthreads=2, lib=lib)
+    of, lf = O.fwd(qfull, k, v, 0.6, True, nthreads=2, lib=lib)
+    _close(o, of[nk - nq:], 1e-13, "cache suffix O")
+    _close(lse, lf[nk - nq:], 1e-13, "cache suffix LSE")
+    dq, dk, dv, _, _ = O.bwd(q, k, v, do, 0.6, True, nthreads=2, lib=lib)
+    dqf, dkf, dvf, _, _ = O.bwd(qfull, k, v, dofull, 0.6, True, nthreads=3, lib=lib)
+    _close(dq, dqf[nk - nq:], 1e-13, "cache suffix dQ")
+    _close(dk, dkf, 1e-13, "cache suffix dK")
+    _close(dv, dvf, 1e-13, "cache suffix dV")
+
+
+def pin_gqa_torch(lib):
+    """Grouped-query attention (Hq query heads over Hkv key/value heads) against torch fp64 with the
+    key/value heads repeated per group: autograd sums the gradients of a repeated head."""
+    import torch
+    for (Hq, Hkv, nq, nk, causal, seed) in ((4, 2, 9, 9, True, 41), (6, 1, 6, 10, True, 42), (4, 4, 7, 7, False, 43),
+                                             (8, 2, 12, 5, False, 44)):
+        d = 6
+        r = _rng(seed)
+        Q, dO = r.standard_normal((Hq, nq, d)), r.standard_normal((Hq, nq, d))
+        K, V = r.standard_normal((Hkv, nk, d)), r.standard_normal((Hkv, nk, d))
+        scale = 1.0 / math.sqrt(d)
+        G = Hq // Hkv
+        t = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V)]
+        i = np.arange(nq)[:, None]; j = np.arange(nk)[None, :]
+        mask = torch.tensor((j <= i + (nk - nq)) if causal else np.ones((nq, nk), bool))
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            t[0], t[1].repeat_interleave(G, dim=0), t[2].repeat_interleave(G, dim=0), attn_mask=mask, scale=scale)
+        ref.backward(torch.tensor(dO))
+        o, _ = O.gqa_fwd(Q, K, V, scale, causal, nthreads=2, lib=lib)
+        _close(o, ref.detach().numpy(), 1e-12, f"GQA O {Hq}/{Hkv}")
+        dq, dk, dv, _, _ = O.gqa_bwd(Q, K, V, dO, scale, causal, nthreads=2, lib=lib)
+        for a, b, nm in ((dq, t[0].grad, "dQ"), (dk, t[1].grad, "dK"), (dv, t[2].grad, "dV")):
+            _close(a, b.numpy(), 1e-11, f"GQA {nm} {Hq}/{Hkv}")
+
+
 PINS = [pin_golden_worked_example, pin_torch_library, pin_zero_query, pin_single_key,
         pin_constant_values, pin_dominant_logit, pin_rows_sum_to_one, pin_key_shift,
         pin_permutation, pin_causal_prefix, pin_gradient_sums, pin_finite_differences,
-        pin_row_subsets]
+        pin_row_subsets, pin_torch_rectangular, pin_cache_suffix, pin_gqa_torch]

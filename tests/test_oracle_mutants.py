@@ -15,7 +15,9 @@ MUTANTS = {
                       "s[j] = dot(qi, J->k + j * J->d, J->d);"),
     "transposed_scores": ("s[j] = J->scale * dot(qi, J->k + j * J->d, J->d);",
                           "s[j] = J->scale * dot(J->q + j * J->d, J->k + i * J->d, J->d);"),
-    "causal_off_by_one": ("return causal ? i + 1 : n;", "return causal ? (i > 0 ? i : 1) : n;"),
+    "causal_off_by_one": ("int64_t v = i + 1 + (nk - nq);", "int64_t v = i + (nk - nq);"),
+    "causal_top_left": ("int64_t v = i + 1 + (nk - nq);", "int64_t v = i + 1;"),
+    "masked_row_sees_a_key": ("return v < 0 ? 0 : (v > nk ? nk : v);", "return v < 1 ? 1 : (v > nk ? nk : v);"),
     "lse_without_max": ("return m + log(l);", "return log(l);"),
     "values_from_keys": ("const double *vj = J->v + j * J->d;\n            for (int64_t c = 0; c < J->d; ++c) o[c] += p * vj[c];",
                          "const double *vj = J->k + j * J->d;\n            for (int64_t c = 0; c < J->d; ++c) o[c] += p * vj[c];"),
@@ -24,7 +26,9 @@ MUTANTS = {
     "dk_wrong_operand": ("dk[c] += dsij * qi[c];", "dk[c] += dsij * doi[c];"),
     "dv_uses_dS": ("dv[c] += p * doi[c];", "dv[c] += dsij * doi[c];"),
     "dk_missing_scale": ("for (int64_t c = 0; c < J->d; ++c) dk[c] *= J->scale;", ""),
-    "dkdv_causal_range": ("int64_t i0 = J->causal ? j : 0;", "int64_t i0 = J->causal ? j + 1 : 0;"),
+    "dkdv_causal_range": ("int64_t i0 = J->causal ? j - (J->nk - J->nq) : 0;",
+                          "int64_t i0 = J->causal ? j + 1 - (J->nk - J->nq) : 0;"),
+    "dkdv_top_left": ("int64_t i0 = J->causal ? j - (J->nk - J->nq) : 0;", "int64_t i0 = J->causal ? j : 0;"),
     "dP_wrong_sign": ("double dsij = p * (dp - J->dsum_all[i]);", "double dsij = p * (J->dsum_all[i] - dp);"),
 }
 
