@@ -25,6 +25,10 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I,
                     ctypes.c_float, _I, _P]),
+    "fa_fwd_qk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
+    "fa_bwd_qk_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "fa_bwd_qk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _I,
+                       ctypes.c_float, _I, _P]),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_last_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "fa_set_softmax_options": (_I, [ctypes.c_float, _I]),

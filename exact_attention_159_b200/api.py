@@ -97,6 +97,60 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, scale: float | None = None, causal: bool
     return dq, dk, dv
 
 
+def _shape_qk(q, k):
+    B, Hq, Nq, d = _shape(q)
+    Bk, Hkv, Nk, dk = _shape(k)
+    if Bk != B or dk != d:
+        raise ValueError("q and k must agree in batch and head dimension")
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def fa_fwd_qk(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None, stream=None):
+    """O, LSE of grouped-query attention with Nq queries over Nk keys: q bf16 [B, Hq, Nq, d],
+    k/v bf16 [B, Hkv, Nk, d] (Hq a multiple of Hkv; causal aligns the last query with the last key)."""
+    B, Hq, Hkv, Nq, Nk, d = _shape_qk(q, k)
+    _need(q, "q", _BF16, (B, Hq, Nq, d))
+    for t, nm in ((k, "k"), (v, "v")):
+        _need(t, nm, _BF16, (B, Hkv, Nk, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", _BF16, (B, Hq, Nq, d))
+    _need(lse, "lse", torch.float32, (B, Hq, Nq))
+    check(_lib.lib().fa_fwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
+                               int(bool(causal)), _stream(stream)), "fa_fwd_qk")
+    return out, lse
+
+
+def fa_bwd_qk_workspace_size(B: int, Hq: int, Nq: int, d: int) -> int:
+    return int(_lib.lib().fa_bwd_qk_workspace_size(B, Hq, Nq, d))
+
+
+def fa_bwd_qk(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False,
+              dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ [B, Hq, Nq, d] and dK, dV [B, Hkv, Nk, d] (summed over each key/value head's query heads)."""
+    B, Hq, Hkv, Nq, Nk, d = _shape_qk(q, k)
+    for t, nm in ((q, "q"), (o, "o"), (do, "do")):
+        _need(t, nm, _BF16, (B, Hq, Nq, d))
+    for t, nm in ((k, "k"), (v, "v")):
+        _need(t, nm, _BF16, (B, Hkv, Nk, d))
+    _need(lse, "lse", torch.float32, (B, Hq, Nq))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    ws_bytes = fa_bwd_qk_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    _need(dq, "dq", _BF16, (B, Hq, Nq, d))
+    for t, nm in ((dk, "dk"), (dv, "dv")):
+        _need(t, nm, _BF16, (B, Hkv, Nk, d))
+    check(_lib.lib().fa_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _stream(stream)), "fa_bwd_qk")
+    return dq, dk, dv
+
+
 def fa_last_device_status(stream=None) -> tuple[int, int]:
     """(status, detail) after synchronising the stream; see include/fa.h."""
     detail = ctypes.c_int(0)

@@ -112,22 +112,28 @@ bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Shape checks shared by forward and backward.  Returns FA_OK, or the error; *empty set for 0-size problems.
-int check_shape(int B, int H, int N, int d, float scale, int causal, bool* empty) {
+// Shape checks shared by forward and backward (Hq query heads over Hkv key/value heads, Nq query
+// and Nk key rows).  Returns FA_OK, or the error; *empty set for 0-size problems.
+int check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, bool* empty) {
   *empty = false;
-  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (B == 0 || H == 0 || N == 0) {
+  if (Hkv == 0 ? Hq != 0 : Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Nq == 0) {
     *empty = true;
     return FA_OK;
   }
-  const long long BH = static_cast<long long>(B) * H;
-  const long long tiles = (static_cast<long long>(N) + 127) / 128;
-  // grid size, tensor-map extents and int row indices must stay in range
-  if (BH > INT_MAX / 2 || BH * tiles > INT_MAX || static_cast<long long>(N) + 128 > INT_MAX) return FA_ERR_UNSUPPORTED;
-  if (BH * (tiles * 128) * d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  if (Nk == 0) return FA_ERR_INVALID_ARG;  // every query needs a key set to attend to
+  for (const long long N : {static_cast<long long>(Nq), static_cast<long long>(Nk)}) {
+    const long long BH = static_cast<long long>(B) * (N == Nq ? Hq : Hkv);
+    const long long tiles = (N + 127) / 128;
+    // grid size, tensor-map extents and int row indices must stay in range
+    if (BH > INT_MAX / 2 || BH * tiles > INT_MAX || N + 128 > INT_MAX) return FA_ERR_UNSUPPORTED;
+    if (BH * (tiles * 128) * d > (1LL << 46)) return FA_ERR_UNSUPPORTED;
+  }
+  if (static_cast<long long>(B) * Hq * ((Nq + 127) / 128) > INT_MAX) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -163,7 +169,7 @@ int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   using L = fa::BwdLayout<D>;
   auto kern = fa::bwd_kernel<D, C, kBwdPoly16>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_tiles);
+  const unsigned grid = static_cast<unsigned>(prm.BHkv) * static_cast<unsigned>(prm.n_kv_tiles);
   kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -235,44 +241,51 @@ int fa_set_softmax_options(float tau, int poly) {
   return FA_OK;
 }
 
-int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
-           float scale, int causal, void* stream) {
+int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int Hq, int Hkv, int Nq,
+              int Nk, int d, float scale, int causal, void* stream) {
   bool empty = false;
-  int rc = check_shape(B, H, N, d, scale, causal, &empty);
+  int rc = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty);
   if (rc != FA_OK) return rc;
   if (!Q || !K || !V || !O || !LSE) return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FA_ERR_ALIGNMENT;
-  const int BH = B * H;
-  const size_t nb = static_cast<size_t>(BH) * N * d * 2, lb = static_cast<size_t>(BH) * N * 4;
-  for (const void* in : {Q, K, V})
-    if (overlaps(O, nb, in, nb) || overlaps(LSE, lb, in, nb)) return FA_ERR_INVALID_ARG;
-  if (overlaps(O, nb, LSE, lb)) return FA_ERR_INVALID_ARG;
+  const int BH = B * Hq, BHkv = B * Hkv;
+  const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, kb = static_cast<size_t>(BHkv) * Nk * d * 2;
+  const size_t lb = static_cast<size_t>(BH) * Nq * 4;
+  const void* ins[3] = {Q, K, V};
+  const size_t isz[3] = {qb, kb, kb};
+  for (int i = 0; i < 3; ++i)
+    if (overlaps(O, qb, ins[i], isz[i]) || overlaps(LSE, lb, ins[i], isz[i])) return FA_ERR_INVALID_ARG;
+  if (overlaps(O, qb, LSE, lb)) return FA_ERR_INVALID_ARG;
   int* status = device_status(&rc);
   if (!status) return rc;
 
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d))
+  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d))
     return FA_ERR_CUDA;
   fa::FwdParams prm;
   prm.O = static_cast<__nv_bfloat16*>(O);
   prm.LSE = LSE;
-  prm.N = N;
+  prm.N = Nq;
+  prm.Nk = Nk;
   prm.BH = BH;
-  const int tiles = (N + 127) / 128;
+  prm.Hq = Hq;
+  prm.G = Hq / Hkv;
+  prm.off = Nk - Nq;
+  const int tiles = (Nq + 127) / 128;
   prm.n_pairs = (tiles + 1) / 2;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.tau = g_tau;
   prm.status = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool poly = g_poly != 0;
-  if (d == 128 && g_fwd_pair) {
+  if (d == 128 && g_fwd_pair && Hq == Hkv && Nq == Nk) {
     CUtensorMap mk64;
-    if (!make_map(&mk64, K, BH, N, d, 64)) return FA_ERR_CUDA;
+    if (!make_map(&mk64, K, BH, Nk, d, 64)) return FA_ERR_CUDA;
     fa::Fwd2Params p2;
     p2.O = prm.O;
     p2.LSE = prm.LSE;
-    p2.N = N;
+    p2.N = Nq;
     p2.BH = BH;
     p2.n_quads = (tiles + 3) / 4;
     p2.scale_log2 = prm.scale_log2;
@@ -302,31 +315,39 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int
   return rc;
 }
 
-size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  bool empty = false;
-  if (check_shape(B, H, N, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
-  return ws_layout(static_cast<long long>(B) * H, N, d).total;
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
+           float scale, int causal, void* stream) {
+  return fa_fwd_qk(Q, K, V, O, LSE, B, H, H, N, N, d, scale, causal, stream);
 }
 
-int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
-           void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
-           int causal, void* stream) {
+size_t fa_bwd_qk_workspace_size(int B, int Hq, int Nq, int d) {
   bool empty = false;
-  int rc = check_shape(B, H, N, d, scale, causal, &empty);
+  if (check_shape(B, Hq, Hq, Nq, Nq, d, 1.0f, 0, &empty) != FA_OK || empty) return 0;
+  return ws_layout(static_cast<long long>(B) * Hq, Nq, d).total;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) { return fa_bwd_qk_workspace_size(B, H, N, d); }
+
+int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+              void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk,
+              int d, float scale, int causal, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty);
   if (rc != FA_OK) return rc;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return FA_ERR_INVALID_ARG;
   if (empty) return FA_OK;
   for (const void* p : {Q, K, V, O, dO, static_cast<const void*>(LSE), static_cast<const void*>(dQ),
                         static_cast<const void*>(dK), static_cast<const void*>(dV), static_cast<const void*>(workspace)})
     if (!aligned16(p)) return FA_ERR_ALIGNMENT;
-  const int BH = B * H;
-  const WsLayout ws = ws_layout(BH, N, d);
+  const int BH = B * Hq, BHkv = B * Hkv;
+  const WsLayout ws = ws_layout(BH, Nq, d);
   if (workspace_bytes < ws.total) return FA_ERR_INVALID_ARG;
-  const size_t nb = static_cast<size_t>(BH) * N * d * 2, lb = static_cast<size_t>(BH) * N * 4;
+  const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, kb = static_cast<size_t>(BHkv) * Nk * d * 2;
+  const size_t lb = static_cast<size_t>(BH) * Nq * 4;
   const void* outs[4] = {dQ, dK, dV, workspace};
-  const size_t osz[4] = {nb, nb, nb, ws.total};
+  const size_t osz[4] = {qb, kb, kb, ws.total};
   const void* ins[6] = {Q, K, V, O, dO, LSE};
-  const size_t isz[6] = {nb, nb, nb, nb, nb, lb};
+  const size_t isz[6] = {qb, kb, kb, qb, qb, lb};
   for (int a = 0; a < 4; ++a) {
     for (int b = 0; b < 6; ++b)
       if (overlaps(outs[a], osz[a], ins[b], isz[b])) return FA_ERR_INVALID_ARG;
@@ -337,22 +358,28 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   if (!status) return rc;
 
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  const int tiles = (N + 127) / 128;
-  const int npad = tiles * 128;
+  const int q_tiles = (Nq + 127) / 128;
+  const int npad = q_tiles * 128;
   float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
   CUtensorMap mq, mk, mv, mdo, macc;
-  if (!make_map(&mq, Q, BH, N, d) || !make_map(&mk, K, BH, N, d) || !make_map(&mv, V, BH, N, d) ||
-      !make_map(&mdo, dO, BH, N, d) || !make_acc_map(&macc, dq_acc, BH, npad, d))
+  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d) ||
+      !make_map(&mdo, dO, BH, Nq, d) || !make_acc_map(&macc, dq_acc, BH, npad, d))
     return FA_ERR_CUDA;
   fa::BwdParams prm;
   prm.nlse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
   prm.ndsum = reinterpret_cast<const float*>(wsb + ws.dsum);
   prm.dK = static_cast<__nv_bfloat16*>(dK);
   prm.dV = static_cast<__nv_bfloat16*>(dV);
-  prm.N = N;
+  prm.N = Nq;
   prm.Npad = npad;
-  prm.BH = BH;
-  prm.n_tiles = tiles;
+  prm.Nk = Nk;
+  prm.BHkv = BHkv;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.off = Nk - Nq;
+  prm.n_q_tiles = q_tiles;
+  prm.n_kv_tiles = (Nk + 127) / 128;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.scale = scale;
   prm.status = status;
@@ -366,11 +393,11 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   if (d == 128)
     fa::bwd_prep_kernel<128><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
                                                         static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                        dq_acc, N, npad, prep_rows);
+                                                        dq_acc, Nq, npad, prep_rows);
   else
     fa::bwd_prep_kernel<64><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
                                                        static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                       dq_acc, N, npad, prep_rows);
+                                                       dq_acc, Nq, npad, prep_rows);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   const bool prof = prof_begin(1, st);
@@ -383,13 +410,20 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   if (prof) prof_end(1, st);
   if (rc != FA_OK) return rc;
 
-  const long long rows = static_cast<long long>(BH) * N;
+  const long long rows = static_cast<long long>(BH) * Nq;
   const unsigned cgrid = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
   if (d == 128)
-    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
   else
-    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, N, npad, rows);
+    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+           void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+           int causal, void* stream) {
+  return fa_bwd_qk(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, workspace_bytes, B, H, H, N, N, d, scale, causal,
+                   stream);
 }
 
 }  // extern "C"
@@ -429,7 +463,7 @@ extern "C" {
 int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                    void* dQ, void* dK, void* dV, int B, int H, int N, int d, float scale, int causal, void* stream) {
   bool empty = false;
-  const int rc0 = check_shape(B, H, N, d, scale, causal, &empty);
+  const int rc0 = check_shape(B, H, H, N, N, d, scale, causal, &empty);
   if (rc0 != FA_OK) return rc0;
   if (!empty && fa_bwd_workspace_size(B, H, N, d) > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
   int rc = FA_OK;

@@ -6,8 +6,10 @@
 // kernels run on the caller's stream:
 //   bwd_prep_kernel    D_i = dO_i . O_i, LSE2_i = LSE_i * log2(e) (+inf on the
 //                      padding rows of the last tile), dQ_acc = 0
-//   bwd_kernel         one CTA per (batch*head, 128-row key tile n), key tile
-//                      stationary, loop over the query tiles m that see it:
+//   bwd_kernel         one CTA per (batch * key/value head, 128-row key tile n),
+//                      key tile stationary, loop over the query tiles m that see
+//                      it, of every query head that reads this key/value head
+//                      (grouped-query attention sums their dK, dV in TMEM):
 //                        S^T  = K_n Q_m^T                 (tcgen05 -> TMEM)
 //                        P^T  = 2^(S^T scale log2e - LSE2) (CUDA cores -> TMEM, bf16)
 //                        dP^T = V_n dO_m^T                (tcgen05 -> TMEM)
@@ -29,11 +31,15 @@
 namespace fa {
 
 struct BwdParams {
-  const float* nlse2;  // [BH, Npad]  -LSE * log2(e), -inf on padding rows
-  const float* ndsum;  // [BH, Npad]  -D_i, 0 on padding rows
-  __nv_bfloat16* dK;   // [BH, N, D]
-  __nv_bfloat16* dV;   // [BH, N, D]
-  int N, Npad, BH, n_tiles;
+  const float* nlse2;  // [B * Hq, Npad]  -LSE * log2(e); -inf on padding rows and rows that see no key
+  const float* ndsum;  // [B * Hq, Npad]  -D_i, 0 on padding rows
+  __nv_bfloat16* dK;   // [B * Hkv, Nk, D]
+  __nv_bfloat16* dV;   // [B * Hkv, Nk, D]
+  int N, Npad;         // query rows per head, padded to whole tiles
+  int Nk;              // key rows per head
+  int BHkv, Hq, Hkv, G;  // batch * key/value heads; heads per batch entry; query heads per key/value head
+  int off;             // Nk - N: query row i sees keys j <= i + off when causal
+  int n_q_tiles, n_kv_tiles;
   float scale_log2;    // scale * log2(e)
   float scale;
   int* status;
@@ -90,10 +96,17 @@ __global__ void __launch_bounds__(384, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int bh, n;  // key tile n = 0 (the most causal work) first, a few heads at a time
-  cta_order(blockIdx.x, prm.BH, prm.n_tiles, bh, n);
-  const int m_begin = CAUSAL ? n : 0;
-  const int n_m = prm.n_tiles - m_begin;      // >= 1
+  int bkv, n;  // key tile n = 0 (the most causal work) first, a few heads at a time
+  cta_order(blockIdx.x, prm.BHkv, prm.n_kv_tiles, bkv, n);
+  // first query tile that sees key tile n: its last row + off reaches the tile's first key
+  int m_begin = 0;
+  if (CAUSAL) {
+    const int r0 = n * kTile - prm.off;  // first query row that sees key n * kTile
+    m_begin = r0 <= 0 ? 0 : r0 / kTile;
+  }
+  const int n_m = prm.n_q_tiles - m_begin;  // >= 1: every real key is seen by the last query row
+  const int n_it = prm.G * n_m;             // (query head of the group, query tile) pairs
+  const int bq0 = (bkv / prm.Hkv) * prm.Hq + (bkv % prm.Hkv) * prm.G;  // first query head of the group
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -136,27 +149,27 @@ __global__ void __launch_bounds__(384, 1)
         prefetch_tmap(&tmdO);
         mbar_expect_tx(kv_full, 2 * T);
         for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(smem + L::kK + c * 16384, &tmK, 64 * c, n * kTile, bh, kv_full);
-          tma_load_3d(smem + L::kV + c * 16384, &tmV, 64 * c, n * kTile, bh, kv_full);
+          tma_load_3d(smem + L::kK + c * 16384, &tmK, 64 * c, n * kTile, bkv, kv_full);
+          tma_load_3d(smem + L::kV + c * 16384, &tmV, 64 * c, n * kTile, bkv, kv_full);
         }
         bool ok = true;
         int q_issued = 0, do_issued = 0;
-        for (int mi = 0; mi < n_m; ++mi) {
-          const int m = m_begin + mi, st = mi & 1;
+        for (int it = 0; it < n_it; ++it) {
+          const int bq = bq0 + it / n_m, m = m_begin + it % n_m, st = it & 1;
           // Q_m, -LSE2_m, -D_m into stage st (two stages)
-          if (!(ok = wait(&q_empty[st], ((mi >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
+          if (!(ok = wait(&q_empty[st], ((it >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
           mbar_expect_tx(&q_full[st], T + 1024);
           for (int c = 0; c < kChunks; ++c)
-            tma_load_3d(smem + L::kQ + st * T + c * 16384, &tmQ, 64 * c, m * kTile, bh, &q_full[st]);
-          const size_t off = static_cast<size_t>(bh) * prm.Npad + static_cast<size_t>(m) * kTile;
+            tma_load_3d(smem + L::kQ + st * T + c * 16384, &tmQ, 64 * c, m * kTile, bq, &q_full[st]);
+          const size_t off = static_cast<size_t>(bq) * prm.Npad + static_cast<size_t>(m) * kTile;
           bulk_load(smem + L::kLse + 512 * st, prm.nlse2 + off, 512, &q_full[st]);
           bulk_load(smem + L::kDsum + 512 * st, prm.ndsum + off, 512, &q_full[st]);
           ++q_issued;
           // dO_m (one stage: free once dV_{m-1} has read it)
-          if (!(ok = wait(do_empty, (mi & 1) ^ 1, g, kSiteBwd | 14))) break;
+          if (!(ok = wait(do_empty, (it & 1) ^ 1, g, kSiteBwd | 14))) break;
           mbar_expect_tx(do_full, T);
           for (int c = 0; c < kChunks; ++c)
-            tma_load_3d(smem + L::kdO + c * 16384, &tmdO, 64 * c, m * kTile, bh, do_full);
+            tma_load_3d(smem + L::kdO + c * 16384, &tmdO, 64 * c, m * kTile, bq, do_full);
           ++do_issued;
         }
         if (!ok) {
@@ -192,13 +205,13 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           issue_s(0);
         }
-        for (int mi = 0; ok && mi < n_m; ++mi) {
-          const int st = mi & 1;
-          const uint32_t ph = mi & 1;
+        for (int it = 0; ok && it < n_it; ++it) {
+          const int st = it & 1;
+          const uint32_t ph = it & 1;
           const uint32_t sQ = sQ0 + st * T;
           // dP^T = V dO^T (its columns hold dQ of the previous tile when aliased)
           if (!(ok = wait(do_full, ph, g, kSiteBwd | 15))) break;
-          if (L::kAliasDQ && mi > 0) {
+          if (L::kAliasDQ && it > 0) {
             if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 4))) break;
           }
           tc_fence_after();
@@ -215,11 +228,11 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk)
             mma_ts(tmem + L::kColDV, tmem + L::kColS + 8 * kk, sdesc_sw128(sdO + kk * 2048, 16384, 1024), idKM,
-                   (mi > 0 || kk > 0) ? 1u : 0u);
+                   (it > 0 || kk > 0) ? 1u : 0u);
           tc_commit(do_empty);
           // S^T of the next query tile (P_m in the S columns has been read by the dV MMA above)
-          if (mi + 1 < n_m) {
-            if (!(ok = wait(&q_full[st ^ 1], ((mi + 1) >> 1) & 1, g, kSiteBwd | 16))) break;
+          if (it + 1 < n_it) {
+            if (!(ok = wait(&q_full[st ^ 1], ((it + 1) >> 1) & 1, g, kSiteBwd | 16))) break;
             tc_fence_after();
             issue_s(st ^ 1);
           }
@@ -230,11 +243,11 @@ __global__ void __launch_bounds__(384, 1)
           for (int kk = 0; kk < kTile / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
             mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
-                   idKM, (mi > 0 || kk > 0) ? 1u : 0u);
+                   idKM, (it > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&q_empty[st]);  // Q_m, -LSE2_m, -D_m no longer needed once these land
           // dQ_m = dS K
-          if (!L::kAliasDQ && mi > 0) {
+          if (!L::kAliasDQ && it > 0) {
             if (!(ok = wait(dq_free, ph ^ 1, g, kSiteBwd | 7))) break;
             tc_fence_after();
           }
@@ -260,13 +273,13 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* sdS = smem + L::kdS;
     const float2 c2 = make_float2(prm.scale_log2, prm.scale_log2);
     bool ok = true;
-    for (int mi = 0; mi < n_m; ++mi) {
-      const int m = m_begin + mi, st = mi & 1;
-      const uint32_t ph = mi & 1;
+    for (int it = 0; it < n_it; ++it) {
+      const int m = m_begin + it % n_m, st = it & 1;
+      const uint32_t ph = it & 1;
       const float4* nl4 = reinterpret_cast<const float4*>(smem + L::kLse + 512 * st);
       const float4* nd4 = reinterpret_cast<const float4*>(smem + L::kDsum + 512 * st);
       // -LSE2_m / -D_m arrive with Q_m (TMA); S^T_m is ready once s_full completes
-      if (!(ok = wait_warp(&q_full[st], (mi >> 1) & 1, g, kSiteBwd | 13))) break;
+      if (!(ok = wait_warp(&q_full[st], (it >> 1) & 1, g, kSiteBwd | 13))) break;
       if (!(ok = wait_warp(s_full, ph, g, kSiteBwd | 8))) break;
       tc_fence_after();
       uint32_t sr[4][32];
@@ -276,7 +289,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
       float p[kTile];
-      const bool diag = CAUSAL && m == n;
+      // causal masking in this pair of tiles: query i (of tile m) does not see key j (of tile n)
+      // when n*128 + j > m*128 + i + off, i.e. i < thr
+      const int thr = (n - m) * kTile + j - prm.off;
+      const bool diag = CAUSAL && n * kTile + kTile - 1 > m * kTile + prm.off;
       const bool edge = diag || (m + 1) * kTile > prm.N;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -297,9 +313,9 @@ __global__ void __launch_bounds__(384, 1)
             } else {
               pv.x = exp2_sfu(x.x);
               pv.y = exp2_sfu(x.y);
-              if (diag) {  // query i < key j is masked
-                if (ii < j) pv.x = 0.0f;
-                if (ii + 1 < j) pv.y = 0.0f;
+              if (diag) {
+                if (ii < thr) pv.x = 0.0f;
+                if (ii + 1 < thr) pv.y = 0.0f;
               }
             }
             p[ii] = pv.x;
@@ -315,7 +331,7 @@ __global__ void __launch_bounds__(384, 1)
 
       if (!(ok = wait_warp(dp_full, ph, g, kSiteBwd | 9))) break;
       tc_fence_after();
-      if (mi > 0) {
+      if (it > 0) {
         if (!(ok = wait_warp(ds_empty, ph ^ 1, g, kSiteBwd | 10))) break;
       }
       uint32_t dp_[2][32];
@@ -361,8 +377,8 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after();
       const int key = n * kTile + j;
-      const bool store = key < prm.N;
-      const size_t rowoff = (static_cast<size_t>(bh) * prm.N + (store ? key : 0)) * D;
+      const bool store = key < prm.Nk;
+      const size_t rowoff = (static_cast<size_t>(bkv) * prm.Nk + (store ? key : 0)) * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = tmem + (which == 0 ? L::kColDK : L::kColDV) + lane_off;
@@ -401,9 +417,9 @@ __global__ void __launch_bounds__(384, 1)
     // wait that can fail (dq_full) is followed by a joint decision, so they leave together.
     int flushed = 0;  // quarter tiles handed to TMA so far
     bool ok = true;
-    for (int mi = 0; mi < n_m; ++mi) {
-      const int m = m_begin + mi;
-      const bool okl = ok && wait_warp(dq_full, mi & 1, g, kSiteBwd | 12);
+    for (int it = 0; it < n_it; ++it) {
+      const int bq = bq0 + it / n_m, m = m_begin + it % n_m;
+      const bool okl = ok && wait_warp(dq_full, it & 1, g, kSiteBwd | 12);
       if (!(ok = group_and(1, 128, okl))) break;
       tc_fence_after();
       uint32_t a[D / 32][32];
@@ -426,7 +442,7 @@ __global__ void __launch_bounds__(384, 1)
         fence_proxy_async();
         named_barrier(1, 128);
         if (leader) {
-          tma_reduce_add_3d(&tmdQacc, 32 * c, m * kTile, bh, buf);
+          tma_reduce_add_3d(&tmdQacc, 32 * c, m * kTile, bq, buf);
           bulk_commit();
         }
       }
@@ -478,7 +494,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
   if (live) {
     if (seg == 0) {
       ndsum[r] = valid ? -acc : 0.0f;
-      nlse2[r] = valid ? -LSE[static_cast<size_t>(bh) * N + i] * 1.4426950408889634f : -INFINITY;
+      const float lse = valid ? LSE[static_cast<size_t>(bh) * N + i] : -INFINITY;
+      nlse2[r] = lse == -INFINITY ? -INFINITY : -lse * 1.4426950408889634f;  // -inf: no key seen, P = 0
     }
     float4* z = reinterpret_cast<float4*>(dq_acc + r * D + seg * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);

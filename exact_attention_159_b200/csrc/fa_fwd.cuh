@@ -31,6 +31,8 @@
 // reduces SFU contention").
 #pragma once
 
+#include <type_traits>
+
 #include "exp2_poly.cuh"
 #include "sm100.cuh"
 
@@ -45,8 +47,11 @@ enum : int { kSiteFwd = 0x100, kSiteBwd = 0x200 };
 struct FwdParams {
   __nv_bfloat16* O;   // [BH, N, D]
   float* LSE;         // [BH, N], natural log
-  int N;
-  int BH;
+  int N;              // query rows per head
+  int Nk;             // key rows per head
+  int BH;             // batch * query heads
+  int Hq, G;          // query heads per batch entry; query heads per key/value head
+  int off;            // Nk - N: query row i sees keys j <= i + off when causal
   int n_pairs;        // ceil(ceil(N / 128) / 2)
   float scale_log2;   // softmax scale * log2(e)
   float tau;          // rescale threshold (log2 units)
@@ -112,12 +117,16 @@ __global__ void __launch_bounds__(640, 1)
   int bh, unit;  // heaviest causal work (the last query tiles) first, a few heads at a time
   cta_order(blockIdx.x, prm.BH, prm.n_pairs, bh, unit);
   const int pair = prm.n_pairs - 1 - unit;
-  const int n_tiles = (prm.N + kTile - 1) / kTile;
-  int nkv[2];
+  const int n_tiles = (prm.N + kTile - 1) / kTile;     // query tiles
+  const int n_kv = (prm.Nk + kTile - 1) / kTile;       // key / value tiles
+  // key / value head of this query head (grouped-query attention: G query heads share one)
+  const int bkv = (bh / prm.Hq) * (prm.Hq / prm.G) + (bh % prm.Hq) / prm.G;
+  int nkv[2];  // key tiles query tile qt sees: those holding a key <= its last row + off
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qt = 2 * pair + t;
-    nkv[t] = qt < n_tiles ? (CAUSAL ? qt + 1 : n_tiles) : 0;
+    const int last_key = qt * kTile + kTile - 1 + prm.off;
+    nkv[t] = qt >= n_tiles ? 0 : !CAUSAL ? n_kv : last_key < 0 ? 0 : min(last_key / kTile + 1, n_kv);
   }
   const int nkv_max = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
 
@@ -151,11 +160,11 @@ __global__ void __launch_bounds__(640, 1)
     regs_dec<kFwdRegsCtl>();
     if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && nkv_max > 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_expect_tx(bar_q, (nkv[1] > 0 ? 2 : 1) * T);
+      mbar_expect_tx(bar_q, ((nkv[0] > 0) + (nkv[1] > 0)) * T);
       for (int t = 0; t < 2; ++t)
         if (nkv[t] > 0)
           for (int c = 0; c < kChunks; ++c)
@@ -169,12 +178,12 @@ __global__ void __launch_bounds__(640, 1)
         if (!(ok = wait(&k_empty[s], ph ^ 1, g, kSiteFwd | 1))) break;
         mbar_expect_tx(&k_full[s], T);
         for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(smem + L::kK + s * T + c * 16384, &tmK, 64 * c, j * kTile, bh, &k_full[s]);
+          tma_load_3d(smem + L::kK + s * T + c * 16384, &tmK, 64 * c, j * kTile, bkv, &k_full[s]);
         ++k_issued;
         if (!(ok = wait(&v_empty[s], ph ^ 1, g, kSiteFwd | 12))) break;
         mbar_expect_tx(&v_full[s], T);
         for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(smem + L::kV + s * T + c * 16384, &tmV, 64 * c, j * kTile, bh, &v_full[s]);
+          tma_load_3d(smem + L::kV + s * T + c * 16384, &tmV, 64 * c, j * kTile, bkv, &v_full[s]);
         ++v_issued;
       }
       if (!ok) {  // let copies already in flight land before the CTA exits
@@ -185,7 +194,7 @@ __global__ void __launch_bounds__(640, 1)
     }
     } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
-    if (lane == 0) {
+    if (lane == 0 && nkv_max > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
       const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
@@ -270,13 +279,14 @@ __global__ void __launch_bounds__(640, 1)
       reg_fence(sr[1]);
       // scores stay in the registers tcgen05.ld wrote (S(c) reads local column c as fp32)
 #define S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
-      const bool edge = (CAUSAL && j == qt) || ((j + 1) * kTile > prm.N);
+      // masking: keys past the end, and (causal) keys beyond the first row's reach
+      const bool edge = (CAUSAL && j * kTile + kTile - 1 > qt * kTile + prm.off) || ((j + 1) * kTile > prm.Nk);
       if (edge) {
         const int key0 = j * kTile + 64 * h;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = key0 + c;
-          if (key >= prm.N || (CAUSAL && key > row)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          if (key >= prm.Nk || (CAUSAL && key > row + prm.off)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
       }
       // row maximum: two chains of 3-input max over this half, then the partner's half
@@ -298,30 +308,41 @@ __global__ void __launch_bounds__(640, 1)
         m_ref = m_new;
       }
       // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 columns at a time)
-      const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
+      // a row that has seen no key yet (m_ref = -inf; causal with N > Nk) has only masked scores
+      const float m_sub = m_ref == -INFINITY ? 0.0f : m_ref;
+      const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_sub, -m_sub);
       float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+      // The two paths are separate code, so the tiles that use the cubic for part of their
+      // exponentials issue no SFU operation for that part (a select between the two would).
+      auto exp_store = [&](auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t pk[16];
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = 32 * cc + 2 * e;
-          const float2 x = __ffma2_rn(make_float2(S(c), S(c + 1)), c2, nm2);
-          float2 p;
-          if (!edge && (e & 7) < POLY16 / 2) {
-            p = exp2_poly2(x);
-          } else {
-            p.x = exp2_sfu(x.x);
-            p.y = exp2_sfu(x.y);
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 * cc + 2 * e;
+            const float2 x = __ffma2_rn(make_float2(S(c), S(c + 1)), c2, nm2);
+            float2 p;
+            if (kPoly && (e & 7) < POLY16 / 2) {
+              p = exp2_poly2(x);
+            } else {
+              p.x = exp2_sfu(x.x);
+              p.y = exp2_sfu(x.y);
+            }
+            if (e & 1)
+              ls1 = __fadd2_rn(ls1, p);
+            else
+              ls0 = __fadd2_rn(ls0, p);
+            pk[e] = pack_bf16x2(p.x, p.y);
           }
-          if (e & 1)
-            ls1 = __fadd2_rn(ls1, p);
-          else
-            ls0 = __fadd2_rn(ls0, p);
-          pk[e] = pack_bf16x2(p.x, p.y);
+          tmem_st16(tS + 32 * h + 16 * cc, pk);
         }
-        tmem_st16(tS + 32 * h + 16 * cc, pk);
-      }
+      };
+      if (POLY16 > 0 && !edge)  // masked (edge) tiles keep exact zeros from the SFU
+        exp_store(std::true_type{});
+      else
+        exp_store(std::false_type{});
 #undef S
       const float2 ls = __fadd2_rn(ls0, ls1);
       l += ls.x + ls.y;
@@ -356,7 +377,7 @@ __global__ void __launch_bounds__(640, 1)
     }
     if (ok && nkv[t] > 0) {
       const float l_row = l + xchg[128 * (h ^ 1) + r];
-      const float inv_l = 1.0f / l_row;
+      const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;  // a row that sees no key: O = 0, LSE = -inf
       const bool store = row < prm.N;
       __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D + (D / 2) * h;
 #pragma unroll
@@ -376,7 +397,14 @@ __global__ void __launch_bounds__(640, 1)
         }
       }
       if (store && h == 0)
-        prm.LSE[static_cast<size_t>(bh) * prm.N + row] = (m_ref + log2f(l_row)) * 0.69314718055994531f;
+        prm.LSE[static_cast<size_t>(bh) * prm.N + row] =
+            l_row > 0.0f ? (m_ref + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+    } else if (nkv[t] == 0 && qt < n_tiles && row < prm.N) {
+      // a query tile no key is visible to (causal, N > Nk): O = 0, LSE = -inf
+      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
+#pragma unroll
+      for (int i = 0; i < D / 16; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (h == 0) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
     }
   }
 

@@ -113,6 +113,18 @@ def attention_inputs(workload: int, B: int, H: int, N: int, d: int, *,
     return out
 
 
+def attention_inputs_qk(workload: int, B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, *,
+                        with_do: bool = False) -> dict:
+    """bf16 bit arrays (uint16) for grouped-query attention with unequal lengths: q (and do)
+    B x Hq x Nq x d, k and v B x Hkv x Nk x d, each i.i.d. N(0, 1) from its own stream."""
+    out = {"q": normal_bf16(seed_for(workload, "q"), (B, Hq, Nq, d)),
+           "k": normal_bf16(seed_for(workload, "k"), (B, Hkv, Nk, d)),
+           "v": normal_bf16(seed_for(workload, "v"), (B, Hkv, Nk, d))}
+    if with_do:
+        out["do"] = normal_bf16(seed_for(workload, "do"), (B, Hq, Nq, d))
+    return out
+
+
 # The five workloads of the FlashAttention-4 evaluation this library is
 # measured on (shapes, causal flag, structure).  Workload 5 is a sweep.
 WORKLOADS = {

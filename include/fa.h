@@ -84,6 +84,43 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            void* dQ, void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
            float scale, int causal, void* stream);
 
+/*
+ * Grouped-query attention and unequal query / key lengths (prefill of new
+ * queries against a cache of earlier keys, the serving use the pages name for
+ * FlashAttention-4 -- "NVIDIA Blackwell: FlashAttention-4 Overcomes Memory
+ * Bottlenecks", body, on SGLang / vLLM prefill; GQA / MQA support is listed
+ * as missing in "NVIDIA's FlashAttention-4: Cementing AI Infrastructure
+ * Dominance in 2025", "Limitations and the Road Ahead").
+ *
+ * Q, O: bf16 [B, Hq, Nq, d]; K, V: bf16 [B, Hkv, Nk, d]; LSE: fp32
+ * [B, Hq, Nq].  Hq must be a multiple of Hkv: query head h reads key/value
+ * head h / (Hq / Hkv) (Hkv = 1 is multi-query attention).  causal: query i
+ * sees keys j <= i + (Nk - Nq), i.e. the last query is aligned with the last
+ * key (for Nq == Nk this is the usual mask of fa_fwd).  A query row that sees
+ * no key at all (causal with Nq > Nk) gets O = 0 and LSE = -inf.  B, Hq or
+ * Nq equal to 0 is an empty problem (FA_OK, nothing launched); Nk = 0 with
+ * queries present is FA_ERR_INVALID_ARG.  Otherwise as fa_fwd (fa_fwd is the
+ * case Hq == Hkv, Nq == Nk).  One kernel launch on `stream`.
+ */
+int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int Hq, int Hkv, int Nq,
+              int Nk, int d, float scale, int causal, void* stream);
+
+/* Workspace of fa_bwd_qk: as fa_bwd_workspace_size for the query side [B, Hq, Nq, d]. */
+size_t fa_bwd_qk_workspace_size(int B, int Hq, int Nq, int d);
+
+/*
+ * Backward of fa_fwd_qk.  Q, O, dO: bf16 [B, Hq, Nq, d]; K, V: bf16
+ * [B, Hkv, Nk, d]; LSE: fp32 [B, Hq, Nq] from fa_fwd_qk (read).  dQ: bf16
+ * [B, Hq, Nq, d]; dK, dV: bf16 [B, Hkv, Nk, d], each the sum over the
+ * Hq / Hkv query heads that read that key/value head (written).  workspace:
+ * at least fa_bwd_qk_workspace_size(B, Hq, Nq, d) bytes.  Rows that see no key
+ * contribute nothing and get dQ = 0.  Otherwise as fa_bwd (fa_bwd is the case
+ * Hq == Hkv, Nq == Nk).
+ */
+int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+              void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk,
+              int d, float scale, int causal, void* stream);
+
 /* Static human-readable text for a status code. */
 const char* fa_strerror(int status);
 
