@@ -146,7 +146,8 @@ template <int D, bool C, int P>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const fa::FwdParams& prm,
                cudaStream_t st) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fwd_kernel<D, C, P>;
+  const bool gen = prm.G != 1 || prm.Nk != prm.N;
+  auto kern = gen ? fa::fwd_kernel<D, C, P, true> : fa::fwd_kernel<D, C, P, false>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BH) * static_cast<unsigned>(prm.n_pairs);
   kern<<<grid, L::kThreads, L::kBytes, st>>>(q, k, v, prm);
@@ -167,7 +168,8 @@ template <int D, bool C>
 int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
                const CUtensorMap& dq_acc, const fa::BwdParams& prm, cudaStream_t st) {
   using L = fa::BwdLayout<D>;
-  auto kern = fa::bwd_kernel<D, C, kBwdPoly16>;
+  const bool gen = prm.G != 1 || prm.Nk != prm.N;
+  auto kern = gen ? fa::bwd_kernel<D, C, kBwdPoly16, true> : fa::bwd_kernel<D, C, kBwdPoly16, false>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BHkv) * static_cast<unsigned>(prm.n_kv_tiles);
   kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);

@@ -73,7 +73,9 @@ struct BwdLayout {
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
 constexpr int kBwdRegsCtl = 80, kBwdRegsP = 240, kBwdRegsDQ = 184;
 
-template <int D, bool CAUSAL, int POLY16>
+// GEN: grouped-query heads and / or Nq != Nk; without it (one query head per key/value head,
+// Nq == Nk) the group and offset terms are compile-time constants.
+template <int D, bool CAUSAL, int POLY16, bool GEN>
 __global__ void __launch_bounds__(384, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -96,17 +98,19 @@ __global__ void __launch_bounds__(384, 1)
   int* abort_flag = reinterpret_cast<int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int off = GEN ? prm.off : 0;
+  const int Nk = GEN ? prm.Nk : prm.N;
   int bkv, n;  // key tile n = 0 (the most causal work) first, a few heads at a time
   cta_order(blockIdx.x, prm.BHkv, prm.n_kv_tiles, bkv, n);
   // first query tile that sees key tile n: its last row + off reaches the tile's first key
   int m_begin = 0;
   if (CAUSAL) {
-    const int r0 = n * kTile - prm.off;  // first query row that sees key n * kTile
-    m_begin = r0 <= 0 ? 0 : r0 / kTile;
+    const int r0 = n * kTile - off;  // first query row that sees key n * kTile
+    m_begin = !GEN ? n : r0 <= 0 ? 0 : r0 / kTile;
   }
-  const int n_m = prm.n_q_tiles - m_begin;  // >= 1: every real key is seen by the last query row
-  const int n_it = prm.G * n_m;             // (query head of the group, query tile) pairs
-  const int bq0 = (bkv / prm.Hkv) * prm.Hq + (bkv % prm.Hkv) * prm.G;  // first query head of the group
+  const int n_m = prm.n_q_tiles - m_begin;      // >= 1: every real key is seen by the last query row
+  const int n_it = GEN ? prm.G * n_m : n_m;     // (query head of the group, query tile) pairs
+  const int bq0 = GEN ? (bkv / prm.Hkv) * prm.Hq + (bkv % prm.Hkv) * prm.G : bkv;  // first query head of the group
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -155,7 +159,7 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         int q_issued = 0, do_issued = 0;
         for (int it = 0; it < n_it; ++it) {
-          const int bq = bq0 + it / n_m, m = m_begin + it % n_m, st = it & 1;
+          const int bq = GEN ? bq0 + it / n_m : bq0, m = GEN ? m_begin + it % n_m : m_begin + it, st = it & 1;
           // Q_m, -LSE2_m, -D_m into stage st (two stages)
           if (!(ok = wait(&q_empty[st], ((it >> 1) & 1) ^ 1, g, kSiteBwd | 1))) break;
           mbar_expect_tx(&q_full[st], T + 1024);
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(384, 1)
     const float2 c2 = make_float2(prm.scale_log2, prm.scale_log2);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int m = m_begin + it % n_m, st = it & 1;
+      const int m = GEN ? m_begin + it % n_m : m_begin + it, st = it & 1;
       const uint32_t ph = it & 1;
       const float4* nl4 = reinterpret_cast<const float4*>(smem + L::kLse + 512 * st);
       const float4* nd4 = reinterpret_cast<const float4*>(smem + L::kDsum + 512 * st);
@@ -291,8 +295,8 @@ __global__ void __launch_bounds__(384, 1)
       float p[kTile];
       // causal masking in this pair of tiles: query i (of tile m) does not see key j (of tile n)
       // when n*128 + j > m*128 + i + off, i.e. i < thr
-      const int thr = (n - m) * kTile + j - prm.off;
-      const bool diag = CAUSAL && n * kTile + kTile - 1 > m * kTile + prm.off;
+      const int thr = GEN ? (n - m) * kTile + j - off : j;
+      const bool diag = CAUSAL && (GEN ? n * kTile + kTile - 1 > m * kTile + off : m == n);
       const bool edge = diag || (m + 1) * kTile > prm.N;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -377,8 +381,8 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       tc_fence_after();
       const int key = n * kTile + j;
-      const bool store = key < prm.Nk;
-      const size_t rowoff = (static_cast<size_t>(bkv) * prm.Nk + (store ? key : 0)) * D;
+      const bool store = key < Nk;
+      const size_t rowoff = (static_cast<size_t>(bkv) * Nk + (store ? key : 0)) * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = tmem + (which == 0 ? L::kColDK : L::kColDV) + lane_off;
@@ -418,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
     int flushed = 0;  // quarter tiles handed to TMA so far
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int bq = bq0 + it / n_m, m = m_begin + it % n_m;
+      const int bq = GEN ? bq0 + it / n_m : bq0, m = GEN ? m_begin + it % n_m : m_begin + it;
       const bool okl = ok && wait_warp(dq_full, it & 1, g, kSiteBwd | 12);
       if (!(ok = group_and(1, 128, okl))) break;
       tc_fence_after();

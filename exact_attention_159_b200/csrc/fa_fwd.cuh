@@ -86,7 +86,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
 constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 104;
 
-template <int D, bool CAUSAL, int POLY16>
+// GEN: grouped-query heads and / or N != Nk; without it (one query head per key/value head,
+// N == Nk) the group and offset terms are compile-time constants.
+template <int D, bool CAUSAL, int POLY16, bool GEN>
 __global__ void __launch_bounds__(640, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
@@ -117,15 +119,17 @@ __global__ void __launch_bounds__(640, 1)
   int bh, unit;  // heaviest causal work (the last query tiles) first, a few heads at a time
   cta_order(blockIdx.x, prm.BH, prm.n_pairs, bh, unit);
   const int pair = prm.n_pairs - 1 - unit;
+  const int Nk = GEN ? prm.Nk : prm.N;
+  const int off = GEN ? prm.off : 0;
   const int n_tiles = (prm.N + kTile - 1) / kTile;     // query tiles
-  const int n_kv = (prm.Nk + kTile - 1) / kTile;       // key / value tiles
+  const int n_kv = (Nk + kTile - 1) / kTile;           // key / value tiles
   // key / value head of this query head (grouped-query attention: G query heads share one)
-  const int bkv = (bh / prm.Hq) * (prm.Hq / prm.G) + (bh % prm.Hq) / prm.G;
+  const int bkv = GEN ? (bh / prm.Hq) * (prm.Hq / prm.G) + (bh % prm.Hq) / prm.G : bh;
   int nkv[2];  // key tiles query tile qt sees: those holding a key <= its last row + off
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qt = 2 * pair + t;
-    const int last_key = qt * kTile + kTile - 1 + prm.off;
+    const int last_key = qt * kTile + kTile - 1 + off;
     nkv[t] = qt >= n_tiles ? 0 : !CAUSAL ? n_kv : last_key < 0 ? 0 : min(last_key / kTile + 1, n_kv);
   }
   const int nkv_max = nkv[0] > nkv[1] ? nkv[0] : nkv[1];
@@ -280,13 +284,13 @@ __global__ void __launch_bounds__(640, 1)
       // scores stay in the registers tcgen05.ld wrote (S(c) reads local column c as fp32)
 #define S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
       // masking: keys past the end, and (causal) keys beyond the first row's reach
-      const bool edge = (CAUSAL && j * kTile + kTile - 1 > qt * kTile + prm.off) || ((j + 1) * kTile > prm.Nk);
+      const bool edge = (CAUSAL && j * kTile + kTile - 1 > qt * kTile + off) || ((j + 1) * kTile > Nk);
       if (edge) {
         const int key0 = j * kTile + 64 * h;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int key = key0 + c;
-          if (key >= prm.Nk || (CAUSAL && key > row + prm.off)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          if (key >= Nk || (CAUSAL && key > row + off)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
       }
       // row maximum: two chains of 3-input max over this half, then the partner's half
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(640, 1)
       }
       // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 columns at a time)
       // a row that has seen no key yet (m_ref = -inf; causal with N > Nk) has only masked scores
-      const float m_sub = m_ref == -INFINITY ? 0.0f : m_ref;
+      const float m_sub = GEN && m_ref == -INFINITY ? 0.0f : m_ref;
       const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_sub, -m_sub);
       float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
       // The two paths are separate code, so the tiles that use the cubic for part of their
