@@ -12,7 +12,9 @@
 //   warps 12..19  the same for query tile 1
 // Every score row is split between two threads (two warps on the same TMEM
 // lane quarter): each takes 64 of the 128 key columns, and the pair agrees on
-// the row maximum through shared memory and a 64-thread named barrier.  Four
+// the row maximum through shared memory and a 64-thread hardware barrier that
+// also ANDs the pair's "every wait succeeded" flags (bar.red.and), so a failed
+// wait makes both warps leave together.  Four
 // softmax warps per SM sub-partition hide the SFU and TMEM latencies.
 // Registers are re-split per warpgroup with setmaxnreg (56 / 104 of the
 // 96 x 640 launched).  The softmax arithmetic uses packed fp32x2 FMA/add.
