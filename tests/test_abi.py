@@ -128,3 +128,36 @@ def test_profile_hook_validation(lib):
     assert lib.fa_profile_next(2, None, None) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_profile_next(0, P, None) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_profile_next(1, None, None) == _lib.FA_OK
+
+
+def test_qk_host_validation(lib):
+    p = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(10)]
+
+    def fwd_qk(B=1, Hq=4, Hkv=2, Nq=128, Nk=256, d=64, scale=0.125, causal=1, ptrs=None):
+        a = list(p[:5])
+        for i, v in (ptrs or {}).items():
+            a[i] = v
+        return lib.fa_fwd_qk(*a, B, Hq, Hkv, Nq, Nk, d, scale, causal, None)
+
+    assert fwd_qk(Hq=3, Hkv=2) == _lib.FA_ERR_INVALID_ARG      # Hq not a multiple of Hkv
+    assert fwd_qk(Hkv=0) == _lib.FA_ERR_INVALID_ARG
+    assert fwd_qk(Hkv=-1) == _lib.FA_ERR_INVALID_ARG
+    assert fwd_qk(Nk=0) == _lib.FA_ERR_INVALID_ARG             # queries with no key set
+    assert fwd_qk(Nk=-3) == _lib.FA_ERR_INVALID_ARG
+    assert fwd_qk(d=96) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd_qk(ptrs={1: MIS}) == _lib.FA_ERR_ALIGNMENT
+    assert fwd_qk(ptrs={3: p[1]}) == _lib.FA_ERR_INVALID_ARG   # O aliases K
+    assert fwd_qk(Nq=0) == _lib.FA_OK and fwd_qk(B=0) == _lib.FA_OK and fwd_qk(Hq=0, Hkv=0) == _lib.FA_OK
+    ws = lib.fa_bwd_qk_workspace_size(1, 4, 128, 64)
+    assert ws == lib.fa_bwd_workspace_size(1, 4, 128, 64) > 0
+
+    def bwd_qk(wsb=ws, Hq=4, Hkv=2, Nk=256, ptrs=None):
+        a = list(p)
+        for i, v in (ptrs or {}).items():
+            a[i] = v
+        return lib.fa_bwd_qk(*a, wsb, 1, Hq, Hkv, 128, Nk, 64, 0.125, 1, None)
+
+    assert bwd_qk(Hq=4, Hkv=3) == _lib.FA_ERR_INVALID_ARG
+    assert bwd_qk(wsb=ws - 1) == _lib.FA_ERR_INVALID_ARG
+    assert bwd_qk(ptrs={7: ctypes.c_void_p(0x200000)}) == _lib.FA_ERR_INVALID_ARG   # dK aliases K
+    assert bwd_qk(ptrs={8: MIS}) == _lib.FA_ERR_ALIGNMENT
