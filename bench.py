@@ -50,16 +50,22 @@ def peaks():
         return dict(burst=1590.0, sustained=1400.0, hbm=6650.0, source="fallback")
 
 
+E2E_CHUNKS = 4  # head chunks of the end-to-end step (copies of one chunk overlap another's kernels)
 KERNEL_SOURCES = ("fa_fwd.cuh", "fa_bwd.cuh", "sm100.cuh", "exp2_poly.cuh")
 
 
 def kernel_source_hash():
-    """SHA-256 over the kernel sources; a stored ncu traffic figure is only valid for the same hash."""
+    """SHA-256 over the kernel sources with comments and blank space removed (the code the
+    compiler sees); a stored ncu traffic figure is only valid for the same hash."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "exact_attention_159_b200", "csrc", name), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "exact_attention_159_b200", "csrc", name)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()
 
 
@@ -239,24 +245,60 @@ def run_gpu(args):
     h2d = sum(host[k].numel() * host[k].element_size() for k in ("q", "k", "v", "do"))
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
 
+    # The heads are independent, so the end-to-end step streams them in chunks: the copy of chunk
+    # c+1's inputs and of chunk c-1's results overlap the kernels of chunk c (copy engines on their
+    # own streams, ordered by events).  Every byte still crosses PCIe inside the timed region.
+    n_chunks = E2E_CHUNKS if (B == 1 and H % E2E_CHUNKS == 0) else 1
+    hc = H // n_chunks
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ws_c = torch.empty(api.fa_bwd_workspace_size(B, hc, N, d), dtype=torch.uint8, device="cuda")
+
+    def heads(t, c):
+        return t[:, c * hc:(c + 1) * hc]
+
+    prev_done = [None] * n_chunks  # chunk c's kernels of the previous step read its device inputs
+    prev_out = [None] * n_chunks   # chunk c's copies to the host of the previous step read its outputs
+
     def e2e_step():
-        for k in ("q", "k", "v", "do"):
-            dev[k].copy_(host[k], non_blocking=True)
-        step()
-        h_out["o"].copy_(o, non_blocking=True)
-        h_out["lse"].copy_(lse, non_blocking=True)
-        h_out["dq"].copy_(dq, non_blocking=True)
-        h_out["dk"].copy_(dk, non_blocking=True)
-        h_out["dv"].copy_(dv, non_blocking=True)
+        ev_in = [torch.cuda.Event() for _ in range(n_chunks)]
+        ev_done = [torch.cuda.Event() for _ in range(n_chunks)]
+        ev_out = [torch.cuda.Event() for _ in range(n_chunks)]
+        for c in range(n_chunks):
+            if prev_done[c] is not None:
+                s_in.wait_event(prev_done[c])
+            with torch.cuda.stream(s_in):
+                for k in ("q", "k", "v", "do"):
+                    heads(dev[k], c).copy_(heads(host[k], c), non_blocking=True)
+                ev_in[c].record(s_in)
+        for c in range(n_chunks):
+            stream.wait_event(ev_in[c])
+            if prev_out[c] is not None:
+                stream.wait_event(prev_out[c])
+            q_, k_, v_, do_ = (heads(dev[x], c) for x in ("q", "k", "v", "do"))
+            o_, lse_ = heads(o, c), heads(lse, c)
+            api.fa_fwd(q_, k_, v_, scale, causal, out=o_, lse=lse_)
+            api.fa_bwd(q_, k_, v_, o_, do_, lse_, scale, causal, dq=heads(dq, c), dk=heads(dk, c), dv=heads(dv, c),
+                       workspace=ws_c)
+            ev_done[c].record(stream)
+            s_out.wait_event(ev_done[c])
+            with torch.cuda.stream(s_out):
+                for k, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                    heads(h_out[k], c).copy_(heads(t, c), non_blocking=True)
+                ev_out[c].record(s_out)
+        prev_done[:] = ev_done
+        prev_out[:] = ev_out
 
     e2e_steps = max(1, min(args.steps, 5))
     e2e_step()
+    stream.wait_stream(s_out)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     e0.record(stream)
+    s_in.wait_event(e0)  # the first copies start inside the timed region
     for _ in range(e2e_steps):
         e2e_step()
+    stream.wait_stream(s_out)  # the timed region ends when the last results are on the host
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -292,7 +334,8 @@ def run_gpu(args):
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "e2e": {"value": round(job_tflops(f_fwd + f_bwd, world, e2e_ms), 2), "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
-                "ms_per_step": round(e2e_ms, 3)},
+                "ms_per_step": round(e2e_ms, 3),
+                "pipeline": f"{n_chunks} head chunks; pinned-host copies overlap the kernels on separate streams"},
         "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
     }
