@@ -151,6 +151,35 @@ def fa_bwd_qk(q, k, v, o, do, lse, scale: float | None = None, causal: bool = Fa
     return dq, dk, dv
 
 
+def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, first: bool = False, stream=None) -> None:
+    """Fold a partial (O bf16 [..., d], LSE fp32 [...]) over one key set into an fp32 accumulator."""
+    d = int(o_part.shape[-1])
+    rows = o_part.numel() // d
+    _need(o_part, "o_part", _BF16, tuple(o_part.shape))
+    _need(o_acc, "o_acc", torch.float32, tuple(o_part.shape))
+    _need(lse_part, "lse_part", torch.float32, tuple(o_part.shape[:-1]))
+    _need(lse_acc, "lse_acc", torch.float32, tuple(o_part.shape[:-1]))
+    check(_lib.lib().fa_lse_merge(_ptr(o_part), _ptr(lse_part), _ptr(o_acc), _ptr(lse_acc), rows, d,
+                                  int(bool(first)), _stream(stream)), "fa_lse_merge")
+
+
+def fa_accumulate_bf16(acc, x, first: bool = False, stream=None) -> None:
+    """acc (fp32) = (0 if first else acc) + x (bf16), elementwise."""
+    _need(acc, "acc", torch.float32, tuple(x.shape))
+    _need(x, "x", _BF16, tuple(x.shape))
+    check(_lib.lib().fa_accumulate_bf16(_ptr(acc), _ptr(x), x.numel(), int(bool(first)), _stream(stream)),
+          "fa_accumulate_bf16")
+
+
+def fa_convert_f32_bf16(x, out=None, stream=None):
+    """bf16 copy of an fp32 tensor (round to nearest even)."""
+    out = torch.empty(x.shape, dtype=_BF16, device=x.device) if out is None else out
+    _need(x, "x", torch.float32, tuple(x.shape))
+    _need(out, "out", _BF16, tuple(x.shape))
+    check(_lib.lib().fa_convert_f32_bf16(_ptr(x), _ptr(out), x.numel(), _stream(stream)), "fa_convert_f32_bf16")
+    return out
+
+
 def fa_last_device_status(stream=None) -> tuple[int, int]:
     """(status, detail) after synchronising the stream; see include/fa.h."""
     detail = ctypes.c_int(0)

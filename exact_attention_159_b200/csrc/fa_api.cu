@@ -14,6 +14,7 @@
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
+#include "fa_merge.cuh"
 
 namespace {
 
@@ -491,6 +492,58 @@ int fa_last_device_status(void* stream, int* detail) {
     return FA_ERR_TIMEOUT;
   }
   return FA_OK;
+}
+
+unsigned elementwise_grid(long long items) {
+  const long long blocks = (items + 255) / 256;
+  return static_cast<unsigned>(blocks < 148 * 16 ? (blocks > 0 ? blocks : 1) : 148 * 16);
+}
+
+int fa_lse_merge(const void* O_part, const float* LSE_part, float* O_acc, float* LSE_acc, int64_t rows, int d,
+                 int first, void* stream) {
+  if (rows < 0 || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (rows == 0) return FA_OK;
+  if (!O_part || !LSE_part || !O_acc || !LSE_acc) return FA_ERR_INVALID_ARG;
+  if (!aligned16(O_part) || !aligned16(O_acc) || (reinterpret_cast<uintptr_t>(LSE_part) & 3u) ||
+      (reinterpret_cast<uintptr_t>(LSE_acc) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (rows > (1LL << 40) / d) return FA_ERR_UNSUPPORTED;
+  const size_t pb = static_cast<size_t>(rows) * d * 2, ab = static_cast<size_t>(rows) * d * 4, lb = rows * 4;
+  if (overlaps(O_acc, ab, O_part, pb) || overlaps(O_acc, ab, LSE_part, lb) || overlaps(LSE_acc, lb, O_part, pb) ||
+      overlaps(LSE_acc, lb, LSE_part, lb) || overlaps(O_acc, ab, LSE_acc, lb))
+    return FA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const unsigned grid = elementwise_grid(rows * (d / 8));
+  if (d == 128)
+    fa::lse_merge_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O_part), LSE_part, O_acc,
+                                                    LSE_acc, rows, first);
+  else
+    fa::lse_merge_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O_part), LSE_part, O_acc,
+                                                   LSE_acc, rows, first);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_accumulate_bf16(float* acc, const void* x, int64_t n, int first, void* stream) {
+  if (n < 0 || (n & 7) || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!acc || !x) return FA_ERR_INVALID_ARG;
+  if (!aligned16(acc) || !aligned16(x)) return FA_ERR_ALIGNMENT;
+  if (overlaps(acc, static_cast<size_t>(n) * 4, x, static_cast<size_t>(n) * 2)) return FA_ERR_INVALID_ARG;
+  fa::accumulate_bf16_kernel<<<elementwise_grid(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      acc, static_cast<const __nv_bfloat16*>(x), n / 8, first);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_convert_f32_bf16(const float* x, void* y, int64_t n, void* stream) {
+  if (n < 0 || (n & 7)) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!x || !y) return FA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return FA_ERR_ALIGNMENT;
+  if (overlaps(x, static_cast<size_t>(n) * 4, y, static_cast<size_t>(n) * 2)) return FA_ERR_INVALID_ARG;
+  fa::convert_f32_bf16_kernel<<<elementwise_grid(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, static_cast<__nv_bfloat16*>(y), n / 8);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_set_forward_variant(int cluster_pair) {

@@ -121,6 +121,33 @@ int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const 
               void* dK, void* dV, void* workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk,
               int d, float scale, int causal, void* stream);
 
+/*
+ * Pieces of ring (context-parallel) attention, where each GPU holds one
+ * chunk of the sequence and the key/value chunks travel around the ring of
+ * GPUs (the pages name multi-card use for long contexts -- "NVIDIA Blackwell:
+ * FlashAttention-4 Overcomes Memory Bottlenecks", body).  Exact attention
+ * over the union of disjoint key sets follows from each set's O and LSE:
+ * with L = ln(exp(LSE_a) + exp(LSE_b)), O = exp(LSE_a - L) O_a +
+ * exp(LSE_b - L) O_b.
+ *
+ * fa_lse_merge folds one partial result (O_part bf16 [rows, d], LSE_part
+ * fp32 [rows], as written by fa_fwd / fa_fwd_qk for the same query rows over
+ * one key set) into an fp32 accumulator O_acc [rows, d] / LSE_acc [rows].
+ * first = 1 initialises the accumulator from the partial (its old contents do
+ * not matter).  A row whose LSE is -inf on one side takes the other side; -inf
+ * on both gives O = 0, LSE = -inf.  d in {64, 128}.  O_part and O_acc 16-byte
+ * aligned, the LSE arrays 4-byte aligned; the accumulator must not overlap the
+ * partial.  One kernel launch on `stream`.
+ */
+int fa_lse_merge(const void* O_part, const float* LSE_part, float* O_acc, float* LSE_acc, int64_t rows, int d,
+                 int first, void* stream);
+
+/* acc (fp32, n) = (first ? 0 : acc) + x (bf16, n); n a multiple of 8, both 16-byte aligned. */
+int fa_accumulate_bf16(float* acc, const void* x, int64_t n, int first, void* stream);
+
+/* y (bf16, n) = x (fp32, n) rounded to nearest even; n a multiple of 8, both 16-byte aligned. */
+int fa_convert_f32_bf16(const float* x, void* y, int64_t n, void* stream);
+
 /* Static human-readable text for a status code. */
 const char* fa_strerror(int status);
 

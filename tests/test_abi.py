@@ -161,3 +161,18 @@ def test_qk_host_validation(lib):
     assert bwd_qk(wsb=ws - 1) == _lib.FA_ERR_INVALID_ARG
     assert bwd_qk(ptrs={7: ctypes.c_void_p(0x200000)}) == _lib.FA_ERR_INVALID_ARG   # dK aliases K
     assert bwd_qk(ptrs={8: MIS}) == _lib.FA_ERR_ALIGNMENT
+
+
+def test_merge_helpers_host_validation(lib):
+    A, A2, L1, L2 = (ctypes.c_void_p(0x100000 * i) for i in (1, 2, 3, 4))
+    assert lib.fa_lse_merge(A, L1, A2, L2, 128, 96, 0, None) == _lib.FA_ERR_UNSUPPORTED
+    assert lib.fa_lse_merge(A, L1, A2, L2, -1, 128, 0, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_lse_merge(A, L1, A2, L2, 128, 128, 2, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_lse_merge(None, L1, A2, L2, 128, 128, 0, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_lse_merge(MIS, L1, A2, L2, 128, 128, 0, None) == _lib.FA_ERR_ALIGNMENT
+    assert lib.fa_lse_merge(A, L1, A, L2, 128, 128, 0, None) == _lib.FA_ERR_INVALID_ARG   # accumulator over the partial
+    assert lib.fa_lse_merge(A, L1, A2, L2, 0, 128, 0, None) == _lib.FA_OK
+    assert lib.fa_accumulate_bf16(A2, A, 12, 0, None) == _lib.FA_ERR_INVALID_ARG         # not a multiple of 8
+    assert lib.fa_accumulate_bf16(A2, MIS, 16, 0, None) == _lib.FA_ERR_ALIGNMENT
+    assert lib.fa_convert_f32_bf16(A, A, 16, None) == _lib.FA_ERR_INVALID_ARG            # overlap
+    assert lib.fa_convert_f32_bf16(A, A2, 0, None) == _lib.FA_OK
