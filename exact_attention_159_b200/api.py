@@ -195,6 +195,10 @@ def fa_set_forward_variant(cluster_pair: int = 0) -> None:
     check(_lib.lib().fa_set_forward_variant(int(cluster_pair)), "fa_set_forward_variant")
 
 
+def fa_set_backward_variant(cluster_pair: int = 0) -> None:
+    check(_lib.lib().fa_set_backward_variant(int(cluster_pair)), "fa_set_backward_variant")
+
+
 def fa_exp2_eval(x: torch.Tensor, mode: int = 0, stream=None) -> torch.Tensor:
     """2^x on the device: mode 0 = cubic software exp2, 1 = SFU ex2."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():

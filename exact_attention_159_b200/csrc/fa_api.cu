@@ -12,6 +12,7 @@
 #include "../../include/fa.h"
 #include "exp2_poly.cuh"
 #include "fa_bwd.cuh"
+#include "fa_bwd2.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd2.cuh"
 #include "fa_merge.cuh"
@@ -34,6 +35,7 @@ DeviceState g_dev[kMaxDevices];
 float g_tau = fa::kRescaleTau;
 int g_poly = 0;  // forward default: SFU only (measured faster on B200 than the 1/4 polynomial share)
 int g_fwd_pair = 0;  // 1: forward at d = 128 on cluster pairs (cta_group::2 UMMA)
+int g_bwd_pair = 0;  // 1: backward at d = 128 on cluster pairs (cta_group::2 UMMA)
 cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // one-shot [fwd|bwd][start|stop]
 
 // Records the pending start event of `which` (if any) on `st`; returns whether one was pending.
@@ -98,15 +100,15 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over the fp32 dQ accumulator [BH, Npad, d]: box 32 (d) x 128 (rows) x 1, 128-byte swizzle
-// (the layout of the backward kernel's staging buffers for its TMA reduce-add).
-bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d) {
+// 3-D map over the fp32 dQ accumulator [BH, Npad, d]: box 32 (d) x `rows` x 1, 128-byte swizzle
+// (the layout of the backward kernels' staging buffers for their TMA reduce-add).
+bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d, int rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(npad),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(npad) * d * 4};
-  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -174,6 +176,17 @@ int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BHkv) * static_cast<unsigned>(prm.n_kv_tiles);
   kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <bool C>
+int launch_bwd2(const CUtensorMap& q, const CUtensorMap& q64, const CUtensorMap& k, const CUtensorMap& v,
+                const CUtensorMap& dO, const CUtensorMap& dO64, const CUtensorMap& dq_acc64, const fa::BwdParams& prm,
+                cudaStream_t st) {
+  auto kern = fa::bwd2_kernel<C>;
+  if (set_smem(kern, fa::Bwd2Layout::kBytes) != cudaSuccess) return FA_ERR_CUDA;
+  const unsigned grid = 2u * static_cast<unsigned>(prm.BHkv) * static_cast<unsigned>((prm.n_kv_tiles + 1) / 2);
+  kern<<<grid, 384, fa::Bwd2Layout::kBytes, st>>>(q, q64, k, v, dO, dO64, dq_acc64, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -404,7 +417,15 @@ int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const 
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   const bool prof = prof_begin(1, st);
-  if (d == 128)
+  if (d == 128 && g_bwd_pair && Hq == Hkv && Nq == Nk) {
+    CUtensorMap mq64, mdo64, macc64;
+    if (!make_map(&mq64, Q, BH, Nq, d, 64) || !make_map(&mdo64, dO, BH, Nq, d, 64) ||
+        !make_acc_map(&macc64, dq_acc, BH, npad, d, 64))
+      rc = FA_ERR_CUDA;
+    else
+      rc = causal ? launch_bwd2<true>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st)
+                  : launch_bwd2<false>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st);
+  } else if (d == 128)
     rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, macc, prm, st)
                 : launch_bwd<128, false>(mq, mk, mv, mdo, macc, prm, st);
   else
@@ -549,6 +570,12 @@ int fa_convert_f32_bf16(const float* x, void* y, int64_t n, void* stream) {
 int fa_set_forward_variant(int cluster_pair) {
   if (cluster_pair != 0 && cluster_pair != 1) return FA_ERR_INVALID_ARG;
   g_fwd_pair = cluster_pair;
+  return FA_OK;
+}
+
+int fa_set_backward_variant(int cluster_pair) {
+  if (cluster_pair != 0 && cluster_pair != 1) return FA_ERR_INVALID_ARG;
+  g_bwd_pair = cluster_pair;
   return FA_OK;
 }
 

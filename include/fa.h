@@ -180,6 +180,19 @@ int fa_set_softmax_options(float tau, int poly);
 int fa_set_forward_variant(int cluster_pair);
 
 /*
+ * Backward kernel selection (process-wide; for A/B comparisons).  0: the
+ * single-CTA kernel.  1: at d = 128, for one query head per key/value head and
+ * Nq == Nk, the backward runs on cluster pairs of SMs that own two adjacent
+ * key tiles ("C. Le Duo de Cuisiniers (2-CTA)", FlashAttention-4 pages): every
+ * MMA is a 2-SM (cta_group::2) UMMA, the query-tile operands are split between
+ * the pair, and dQ of a query tile is summed over both key tiles on chip
+ * (each CTA hands the other half of its dS).  Same results, currently slower
+ * (0 is the default); other shapes always use the single-CTA kernel.
+ * Returns FA_ERR_INVALID_ARG for other values.
+ */
+int fa_set_backward_variant(int cluster_pair);
+
+/*
  * Elementwise y = 2^x on the device for testing the exponential the kernels
  * use: mode 0 = the cubic-polynomial software exp2, mode 1 = the SFU
  * (ex2.approx), mode 2 = the cubic with packed fp32x2 arithmetic on element

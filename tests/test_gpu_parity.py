@@ -210,3 +210,41 @@ def test_forward_variants_agree_at_full_size():
         api.fa_set_forward_variant(0)
     assert float((o0.float() - o1.float()).abs().max()) <= 1e-2
     assert float((l0 - l1).abs().max()) <= 1e-3
+
+
+# ----------------------------------------------- backward kernel variants
+# (B, H, N, causal): one key tile (the pair's second tile lies past the end), odd and even tile
+# counts, ragged tails, and several heads and batches
+BWD_VARIANT_SHAPES = [(1, 1, 17, True), (1, 1, 128, True), (1, 2, 200, False), (1, 2, 256, True),
+                      (2, 3, 640, False), (1, 2, 640, True), (1, 4, 1000, True), (1, 2, 1536, False),
+                      (2, 2, 2048, True)]
+
+
+@pytest.mark.parametrize("variant", [0, 1], ids=["single-cta", "cluster-pair"])
+@pytest.mark.parametrize("B,H,N,causal", BWD_VARIANT_SHAPES,
+                         ids=[f"B{b}H{h}N{n}{'c' if c else 'f'}" for b, h, n, c in BWD_VARIANT_SHAPES])
+def test_backward_variants_full(variant, B, H, N, causal):
+    c = Case(B, H, N, 128, causal, seed_workload=15, bwd=True)
+    o, lse = c.fwd_gpu()
+    api.fa_set_backward_variant(variant)
+    try:
+        grads = c.bwd_gpu(o, lse)
+    finally:
+        api.fa_set_backward_variant(0)
+    full = N <= 1000
+    check_bwd(c, grads, all_heads(c), None if full else 96, None if full else 96,
+              f"bwd variant {variant} B{B} H{H} N{N} c{int(causal)}")
+
+
+def test_backward_variants_agree_at_full_size():
+    c = Case(1, 16, 32768, 128, True, seed_workload=4, bwd=True)
+    o, lse = c.fwd_gpu()
+    g0 = c.bwd_gpu(o, lse)
+    api.fa_set_backward_variant(1)
+    try:
+        g1 = c.bwd_gpu(o, lse)
+    finally:
+        api.fa_set_backward_variant(0)
+    check_bwd(c, g1, [(0, 0), (0, 11)], 64, 64, "bwd cluster-pair causal B1 H16 N32768")
+    for a, b in zip(g0, g1):
+        assert rel_l2(b.double().cpu().numpy(), a.double().cpu().numpy()) <= TOL_GRAD
