@@ -18,7 +18,7 @@
 // tensor memory, and the dQ drain (TMEM -> shared memory -> TMA reduce-add) moves half as much
 // per SM: about 350 KB of shared-memory traffic per SM and query tile instead of about 510 KB.
 // Measured on B200 it is nevertheless slower than the single-CTA kernel (the pair instructions
-// of N = 128 run at 100-150 clocks each in situ, the M = 128 dQ instructions at about 140, and
+// of N = 128 run at about 100 clocks each in situ, the M = 128 dQ instructions at about 140, and
 // the remote dS stores with their release cost the dS warps 2,000-3,000 clocks per tile), so it
 // is selected only on request.
 //
@@ -208,48 +208,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         constexpr uint32_t idKK = idesc_bf16_f32(256, 128, false, false);  // S^T, dP^T
         constexpr uint32_t idKM = idesc_bf16_f32(256, D, false, true);     // dV, dK: A in TMEM, B MN-major
         constexpr uint32_t idQ = idesc_bf16_f32(128, D, true, true);       // dQ: M = 128 over the pair
-        const uint32_t s0 = smem_u32(smem);  // operand addresses are s0 + compile-time offsets
-        const uint32_t sK = s0 + L::kK, sV = s0 + L::kV, sQS = s0 + L::kQS, sdO = s0 + L::kdO;
+        // Descriptors: one base per operand buffer, opaque to the compiler inside each query tile
+        // (so it neither hoists a descriptor per instruction nor recomputes them one by one); each
+        // instruction adds its compile-time offset (bytes / 16) to the address field.
+        const uint32_t s0 = smem_u32(smem);
+        auto base = [&](uint32_t off, uint32_t lbo) {
+          uint64_t d = sdesc_sw128(s0 + off, lbo, 1024);
+          asm volatile("" : "+l"(d));
+          return d;
+        };
         // S^T or dP^T: A = own K or V (column block b at b * 16K), B = this CTA's 64 query rows
         // (column block b at b * 8K)
-        auto issue_rows = [&](uint32_t d_col, uint32_t sA, uint32_t sB) {
-#pragma unroll 1
+        auto issue_rows = [&](uint32_t d_col, uint64_t dA, uint64_t dB) {
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t b = kk >> 2, k16 = (kk & 3) * 32;
-            mma_ss_pair(tmem + d_col, sdesc_sw128(sA + b * L::kBlock + k16, 16, 1024),
-                        sdesc_sw128(sB + b * L::kHalf + k16, 16, 1024), idKK, kk > 0);
+            mma_ss_pair(tmem + d_col, dA + ((b * L::kBlock + k16) >> 4), dB + ((b * L::kHalf + k16) >> 4), idKK,
+                        kk > 0);
           }
         };
         bool ok = wait(kv_full, 0, g, kSiteBwd | 0x33) && wait(qs_full, 0, g, kSiteBwd | 0x34);
         if (ok) {
           tc_fence_after();
-          issue_rows(L::kColS, sK, sQS);
+          issue_rows(L::kColS, base(L::kK, 16), base(L::kQS, 16));
           tc_commit_pair(s_full);
           tc_commit_pair(qs_empty);
         }
         for (int it = 0; ok && it < n_it; ++it) {
           const int st = it & 1;
           const uint32_t ph = it & 1;
-          const uint32_t sQK = s0 + L::kQK + st * L::kBlock;
           // dP^T = V dO^T (its last 64 columns hold dQ of the previous tile)
           if (!(ok = wait(do_full, ph, g, kSiteBwd | 0x35))) break;
           if (it > 0 && !(ok = wait_cluster(dq_free, ph ^ 1, g, kSiteBwd | 0x36))) break;
           tc_fence_after();
-          issue_rows(L::kColDP, sV, sdO + L::kBlock);
+          issue_rows(L::kColDP, base(L::kV, 16), base(L::kdO + L::kBlock, 16));
           tc_commit_pair(dp_full);
           // dV += P^T dO (B: all query rows of column block r)
           if (!(ok = wait_cluster(p_full, ph, g, kSiteBwd | 0x37))) break;
           tc_fence_after();
-#pragma unroll 1
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts_pair(tmem + L::kColDV, tmem + L::kColS + 8 * kk, sdesc_sw128(sdO + kk * 2048, L::kBlock, 1024),
-                        idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          {
+            const uint64_t dB = base(L::kdO, L::kBlock);
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts_pair(tmem + L::kColDV, tmem + L::kColS + 8 * kk, dB + ((kk * 2048) >> 4), idKM,
+                          (it > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit_pair(do_empty);
           // S^T of the next query tile (P_m in the S columns has been read by the dV MMA above)
           if (it + 1 < n_it) {
             if (!(ok = wait(qs_full, (it + 1) & 1, g, kSiteBwd | 0x38))) break;
             tc_fence_after();
-            issue_rows(L::kColS, sK, sQS);
+            issue_rows(L::kColS, base(L::kK, 16), base(L::kQS, 16));
             tc_commit_pair(s_full);
             tc_commit_pair(qs_empty);
           }
@@ -257,19 +266,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           if (!(ok = wait_cluster(dst_full, ph, g, kSiteBwd | 0x39))) break;
           if (!(ok = wait(&q_full[st], (it >> 1) & 1, g, kSiteBwd | 0x41))) break;
           tc_fence_after();
-#pragma unroll 1
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            mma_ts_pair(tmem + L::kColDK, tmem + L::kColDP + 8 * kk, sdesc_sw128(sQK + kk * 2048, L::kBlock, 1024),
-                        idKM, (it > 0 || kk > 0) ? 1u : 0u);
+          {
+            const uint64_t dB = base(L::kQK + st * L::kBlock, L::kBlock);
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts_pair(tmem + L::kColDK, tmem + L::kColDP + 8 * kk, dB + ((kk * 2048) >> 4), idKM,
+                          (it > 0 || kk > 0) ? 1u : 0u);
+          }
           tc_commit_pair(&q_empty[st]);
           // dQ_m = dS K over both key tiles of the pair (K-dimension: the keys of n0, then of n1)
           if (!(ok = wait_cluster(dss_full, ph, g, kSiteBwd | 0x3A))) break;
           tc_fence_after();
-#pragma unroll 1
-          for (int kk = 0; kk < 2 * kTile / 16; ++kk) {
-            const uint32_t off = (kk & 7) * 2048;
-            mma_ss_pair(tmem + L::kColDQ, sdesc_sw128(s0 + (kk < 8 ? L::kDSX : L::kDSY) + off, L::kBlock, 1024),
-                        sdesc_sw128(s0 + (kk < 8 ? L::kKX : L::kKY) + off, L::kBlock, 1024), idQ, kk > 0);
+          {
+            const uint64_t dA = base(L::kDSX, L::kBlock), dB = base(L::kKX, L::kBlock);
+#pragma unroll
+            for (int kk = 0; kk < 2 * kTile / 16; ++kk) {
+              const uint32_t off = (kk >> 3) * L::kBlock + (kk & 7) * 2048;  // DSY / KY follow DSX / KX
+              mma_ss_pair(tmem + L::kColDQ, dA + (off >> 4), dB + (off >> 4), idQ, kk > 0);
+            }
           }
           tc_commit_pair(dq_full);
           tc_commit_pair(ds_empty);
