@@ -13,17 +13,20 @@
 //                        S^T  = K_n Q_m^T                 (tcgen05 -> TMEM)
 //                        P^T  = 2^(S^T scale log2e - LSE2) (CUDA cores -> TMEM, bf16)
 //                        dP^T = V_n dO_m^T                (tcgen05 -> TMEM)
-//                        dS^T = P^T (dP^T - D)            (CUDA cores -> smem, bf16)
+//                        dS^T = P^T (dP^T - D)            (CUDA cores -> smem and TMEM, bf16)
 //                        dV  += P^T dO_m                  (A from TMEM)
-//                        dK  += dS^T Q_m
-//                        dQ_m = dS K_n                    (TMEM) -> fp32 atomics into dQ_acc
+//                        dK  += dS^T Q_m                  (A from TMEM)
+//                        dQ_m = dS K_n                    (A from smem; TMEM) -> fp32 TMA reduce-add
+//                                                          into dQ_acc
 //                      dK (x scale) and dV leave TMEM once, at the end.
 //   bwd_dq_kernel      dQ = bf16(scale * dQ_acc)
 // Warps: 0 TMA producer, 1 MMA issuer + TMEM owner, 2..5 P/dS for the 128 key
 // rows (thread = key row), 6..9 dQ drain (thread = query row).
 // Tensor memory columns: dK [0,D), dV [D,2D), S^T [2D,2D+128),
-// dP^T [2D+128,2D+256); dQ reuses the dP^T columns when D = 128 (the 512
-// columns are otherwise full) and has its own 64 columns when D = 64.
+// dP^T [2D+128,2D+256) with dS^T (bf16, packed two per column) written over
+// its first 64 columns once they have been read; dQ reuses the dP^T columns
+// when D = 128 (the 512 columns are otherwise full; dK, issued first, has read
+// dS^T by then) and has its own 64 columns when D = 64.
 #pragma once
 
 #include "fa_fwd.cuh"
@@ -240,15 +243,13 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after();
             issue_s(st ^ 1);
           }
-          // dK += dS^T Q
+          // dK += dS^T Q (dS^T from TMEM, over the dP^T columns)
           if (!(ok = wait(ds_full, ph, g, kSiteBwd | 6))) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + L::kColDK, sdesc_sw128(sdS + off, 16, 1024), sdesc_sw128(sQ + kk * 2048, 16384, 1024),
-                   idKM, (it > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            mma_ts(tmem + L::kColDK, tmem + L::kColDP + 8 * kk, sdesc_sw128(sQ + kk * 2048, 16384, 1024), idKM,
+                   (it > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&q_empty[st]);  // Q_m, -LSE2_m, -D_m no longer needed once these land
           // dQ_m = dS K
           if (!L::kAliasDQ && it > 0) {
@@ -365,6 +366,8 @@ __global__ void __launch_bounds__(384, 1)
           w[2 * e4 + 1] = pack_bf16x2(d1.x, d1.y);
         }
         // columns 32c .. 32c+31 live in chunk (32c / 64), 16-byte groups 4*(c&1) .. +3
+        // dS^T to TMEM for dK, over dP^T columns already read (block c lands in columns 16c..16c+15)
+        tmem_st16(tdP + 16 * c, w);
         uint8_t* base = sdS + (c >> 1) * 16384;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -374,6 +377,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       fence_proxy_async();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(ds_full);
     }

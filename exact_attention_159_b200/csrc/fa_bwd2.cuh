@@ -14,9 +14,8 @@
 //                        hands the other the half of its dS^T that the other's query rows need
 //                        (shared memory of the peer, written directly), so dQ of a query tile
 //                        is summed over two key tiles before it leaves the chip
-// Against the single-CTA kernel every B operand is read half by each SM, dS^T feeds dK from
-// tensor memory, and the dQ drain (TMEM -> shared memory -> TMA reduce-add) moves half as much
-// per SM: about 350 KB of shared-memory traffic per SM and query tile instead of about 510 KB.
+// Against the single-CTA kernel every B operand is read half by each SM, and the dQ drain (TMEM -> shared memory -> TMA reduce-add) moves half as much
+// per SM: about 350 KB of shared-memory traffic per SM and query tile instead of about 500 KB.
 // Measured on B200 it is nevertheless slower than the single-CTA kernel (the pair instructions
 // of N = 128 run at about 100 clocks each in situ, the M = 128 dQ instructions at about 140, and
 // the remote dS stores with their release cost the dS warps 2,000-3,000 clocks per tile), so it
