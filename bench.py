@@ -51,6 +51,7 @@ def peaks():
 
 
 E2E_CHUNKS = 4  # head chunks of the end-to-end step (copies of one chunk overlap another's kernels)
+PROBE_STEPS, PROBE_KEEP = 24, 16  # untimed steps with clock probes after the timed loop; kept (last)
 KERNEL_SOURCES = ("fa_fwd.cuh", "fa_bwd.cuh", "sm100.cuh", "exp2_poly.cuh")
 
 
@@ -239,6 +240,23 @@ def run_gpu(args):
     fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
     bwd_ms = [e[2].elapsed_time(e[3]) for e in ev]
 
+    # The SM clock the kernels actually ran at, measured on the device right after the timed loop
+    # (untimed): a probe kernel queued behind the forward and the backward of a few more steps,
+    # with no synchronisation in between (an idle gap lets the power manager raise the clock).
+    # Under the power cap it can sit well below what nvidia-smi's sampled clocks.sm reports.
+    # The host work after the loop idles the GPU long enough for the clock to recover, so the pass
+    # runs PROBE_STEPS steps and keeps the last PROBE_KEEP, once the power manager has settled.
+    probe = torch.zeros((2 * PROBE_STEPS, 2), dtype=torch.int64, device="cuda")
+    for i in range(PROBE_STEPS):
+        api.fa_fwd(dev["q"], dev["k"], dev["v"], scale, causal, out=o, lse=lse)
+        api.fa_sm_clock_probe(probe[2 * i], stream)
+        api.fa_bwd(dev["q"], dev["k"], dev["v"], o, dev["do"], lse, scale, causal, dq=dq, dk=dk, dv=dv,
+                   workspace=ws)
+        api.fa_sm_clock_probe(probe[2 * i + 1], stream)
+    torch.cuda.synchronize()
+    eff_all = [1000.0 * c / ns if ns > 0 else 0.0 for c, ns in probe.tolist()]
+    eff_mhz = [x for x in eff_all[-2 * PROBE_KEEP:] if x > 0]
+
     # end to end through host buffers
     h_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in
              (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
@@ -337,7 +355,11 @@ def run_gpu(args):
                 "ms_per_step": round(e2e_ms, 3),
                 "pipeline": f"{n_chunks} head chunks; pinned-host copies overlap the kernels on separate streams"},
         "gpu_launches": 4 * args.steps,
-        "clocks": clk.summary(),
+        "clocks": {**clk.summary(), "sm_mhz_effective": round(statistics.median(eff_mhz)) if eff_mhz else None,
+                   "sm_mhz_effective_range": [round(min(eff_mhz)), round(max(eff_mhz))] if eff_mhz else None,
+                   "sm_mhz_effective_how": f"device probe (clock64 cycles over 20 us of %globaltimer) queued behind "
+                                           f"the forward and the backward of the last {PROBE_KEEP} of {PROBE_STEPS} "
+                                           f"untimed steps run back to back after the timed loop"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)

@@ -39,6 +39,7 @@ SIGNATURES = {
     "fa_profile_next": (_I, [_I, _P, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float, _I, _P]),
     "fa_selftest_wait_timeout": (_I, [_P]),
+    "fa_sm_clock_probe": (_I, [_P, _P]),
     "fa_set_forward_variant": (_I, [_I]),
     "fa_set_backward_variant": (_I, [_I]),
     "fa_version": (_I, []),

@@ -214,6 +214,24 @@ def fa_profile_next(which: int, start, stop) -> None:
     check(_lib.lib().fa_profile_next(int(which), h(start), h(stop)), "fa_profile_next")
 
 
+def fa_sm_clock_probe(out: torch.Tensor | None = None, stream=None):
+    """Effective SM clock, measured on the device by a ~20 us probe kernel queued on `stream`
+    behind whatever work is already queued there.  With `out` (a CUDA int64 tensor of 2 elements)
+    it only queues the probe, which writes [cycles, nanoseconds] there (no synchronisation, so
+    the GPU keeps the clock of the surrounding work); without, it synchronises and returns MHz."""
+    own = out is None
+    if own:
+        out = torch.zeros(2, dtype=torch.int64, device="cuda")
+    elif out.dtype != torch.int64 or not out.is_cuda or out.numel() != 2 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CUDA int64 tensor of 2 elements")
+    check(_lib.lib().fa_sm_clock_probe(_ptr(out), _stream(stream)), "fa_sm_clock_probe")
+    if not own:
+        return None
+    torch.cuda.synchronize()
+    cycles, ns = out.tolist()
+    return 1000.0 * cycles / ns if ns > 0 else 0.0
+
+
 def fa_strerror(code: int) -> str:
     return _lib.lib().fa_strerror(int(code)).decode()
 

@@ -220,6 +220,17 @@ __global__ void selftest_wait_kernel(int* status) {
   if (threadIdx.x == 0) fa::mbar_arrive(&bar);  // complete the phase so the barrier is left idle
 }
 
+// One thread: SM cycles elapsed while the global timer advances by 20 us (a bounded spin).
+__global__ void clock_probe_kernel(unsigned long long* out) {
+  const unsigned long long t0 = fa::globaltimer();
+  const long long c0 = clock64();
+  unsigned long long t1 = t0;
+  while (t1 - t0 < 20000ull) t1 = fa::globaltimer();
+  const long long c1 = clock64();
+  out[0] = static_cast<unsigned long long>(c1 - c0);
+  out[1] = t1 - t0;
+}
+
 __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int mode) {
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
@@ -584,6 +595,13 @@ int fa_profile_next(int which, void* start_event, void* stop_event) {
   g_prof[which][0] = static_cast<cudaEvent_t>(start_event);
   g_prof[which][1] = static_cast<cudaEvent_t>(stop_event);
   return FA_OK;
+}
+
+int fa_sm_clock_probe(uint64_t* out, void* stream) {
+  if (!out) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) & 7u) return FA_ERR_ALIGNMENT;
+  clock_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<unsigned long long*>(out));
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_selftest_wait_timeout(void* stream) {

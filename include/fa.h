@@ -212,6 +212,17 @@ int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
 int fa_profile_next(int which, void* start_event, void* stop_event);
 
 /*
+ * SM clock probe (used by the benchmark to state the clock the kernels ran
+ * at): launches one single-thread kernel on `stream` that counts SM cycles
+ * (clock64) while the global nanosecond timer advances by about 20 us, and
+ * writes out[0] = cycles, out[1] = nanoseconds; the effective SM clock is
+ * 1000 * out[0] / out[1] MHz at the moment the probe runs (for example right
+ * after an attention kernel, before the power manager reacts).  `out` is a
+ * device array of two uint64, 8-byte aligned.  Returns the launch status.
+ */
+int fa_sm_clock_probe(uint64_t* out, void* stream);
+
+/*
  * Failure-path self test: launches one small kernel on `stream` whose only
  * pipeline wait is on a barrier that nothing ever arrives at.  The bounded
  * wait used by every kernel of the library gives up after its limit (2 s),

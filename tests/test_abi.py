@@ -176,3 +176,10 @@ def test_merge_helpers_host_validation(lib):
     assert lib.fa_accumulate_bf16(A2, MIS, 16, 0, None) == _lib.FA_ERR_ALIGNMENT
     assert lib.fa_convert_f32_bf16(A, A, 16, None) == _lib.FA_ERR_INVALID_ARG            # overlap
     assert lib.fa_convert_f32_bf16(A, A2, 0, None) == _lib.FA_OK
+
+
+def test_variant_and_probe_host_validation(lib):
+    assert lib.fa_set_backward_variant(2) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_set_backward_variant(-1) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_sm_clock_probe(None, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_sm_clock_probe(ctypes.c_void_p(0x100004), None) == _lib.FA_ERR_ALIGNMENT
