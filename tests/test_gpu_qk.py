@@ -115,3 +115,20 @@ def test_gqa_equals_repeated_heads():
     vr = c.dev["v"].repeat_interleave(c.G, dim=1).contiguous()
     o2, l2 = api.fa_fwd(c.dev["q"], kr, vr, c.scale, True)
     assert torch.equal(o, o2) and torch.equal(lse, l2)
+
+
+@pytest.mark.parametrize("Hq,Hkv,Nq,Nk,d", [(4, 2, 300, 300, 128), (2, 2, 200, 456, 128), (2, 2, 300, 300, 64)],
+                         ids=["gqa", "nq-ne-nk", "d64"])
+def test_backward_pair_switch_leaves_other_shapes_to_the_single_cta_kernel(Hq, Hkv, Nq, Nk, d):
+    # the cluster-pair backward covers d = 128, Hq == Hkv, Nq == Nk only; with it selected, every
+    # other shape still runs (and equals) the single-CTA kernel
+    c = QKCase(1, Hq, Hkv, Nq, Nk, d, True, seed=61)
+    o, lse = api.fa_fwd_qk(c.dev["q"], c.dev["k"], c.dev["v"], c.scale, True)
+    g0 = api.fa_bwd_qk(c.dev["q"], c.dev["k"], c.dev["v"], o, c.dev["do"], lse, c.scale, True)
+    api.fa_set_backward_variant(1)
+    try:
+        g1 = api.fa_bwd_qk(c.dev["q"], c.dev["k"], c.dev["v"], o, c.dev["do"], lse, c.scale, True)
+    finally:
+        api.fa_set_backward_variant(0)
+    assert torch.equal(g0[1], g1[1]) and torch.equal(g0[2], g1[2])   # dK, dV: same kernel, same bits
+    assert float((g0[0].float() - g1[0].float()).abs().max()) <= 2.0 ** -6 * float(g0[0].float().abs().max())
