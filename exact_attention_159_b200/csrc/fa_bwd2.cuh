@@ -14,12 +14,13 @@
 //                        hands the other the half of its dS^T that the other's query rows need
 //                        (shared memory of the peer, written directly), so dQ of a query tile
 //                        is summed over two key tiles before it leaves the chip
-// Against the single-CTA kernel every B operand is read half by each SM, and the dQ drain (TMEM -> shared memory -> TMA reduce-add) moves half as much
-// per SM: about 350 KB of shared-memory traffic per SM and query tile instead of about 500 KB.
-// Measured on B200 it is nevertheless slower than the single-CTA kernel (the pair instructions
-// of N = 128 run at about 100 clocks each in situ, the M = 128 dQ instructions at about 140, and
-// the remote dS stores with their release cost the dS warps 2,000-3,000 clocks per tile), so it
-// is selected only on request.
+// Against the single-CTA kernel every B operand is read half by each SM, and the dQ drain
+// (TMEM -> shared memory -> TMA reduce-add) moves half as much per SM: about 350 KB of
+// shared-memory traffic per SM and query tile instead of about 500 KB.  Measured on B200 it is
+// nevertheless slower than the single-CTA kernel: at N = 128 the 16 M = 128 dQ instructions cost
+// more than the single-CTA kernel's 8, and the remote dS stores with their release cost the dS
+// warps 2,000-3,000 clocks per tile, on which the MMA issuer then waits.  It is selected only on
+// request.
 //
 // Operand placement.  In a pair MMA the rows of A come half from each CTA while B is one matrix
 // split by columns between the two, so every slice of the contraction must hold the same
