@@ -14,7 +14,9 @@ The backward sends each key/value chunk around the ring once more, together with
 accumulators of its dK and dV: every rank adds the gradients of its queries' attention to
 the chunk it holds (``fa_bwd`` with the global O and LSE of its rows, which make the
 per-chunk pieces exact), keeps its own dQ in fp32, and after the last step hands each
-chunk's accumulators back to the chunk's owner.
+chunk's accumulators back to the chunk's owner.  Both transfers overlap compute: the next
+key/value chunk travels while a step computes, and a chunk's accumulators travel while the
+receiving rank computes its gradients for that chunk, which it adds once they have arrived.
 
 The pages name multi-card use of the kernels for long contexts ("NVIDIA Blackwell:
 FlashAttention-4 Overcomes Memory Bottlenecks", body); the exchange itself is the
@@ -88,17 +90,22 @@ class _BwdState:
         self.dq_acc, self.first = be.f32_like(q), True
 
 
-def _bwd_step(be, st, r, s, world, q, k, v, o, do, lse, dk_acc, dv_acc, scale, causal):
-    """Adds rank r's contributions to dQ and to the held chunk's dK, dV accumulators."""
-    src = source(r, s, world)
-    kind = block_kind(r, src, causal)
-    if kind is not None:
-        dq_p, dk_p, dv_p = be.bwd(q, k, v, o, do, lse, scale, kind == "diag")
-        be.accumulate(st.dq_acc, dq_p, st.first)
-        st.first = False
-        # the chunk's own rank starts its accumulators at step 0 (its diagonal block is never skipped)
-        be.accumulate(dk_acc, dk_p, s == 0)
-        be.accumulate(dv_acc, dv_p, s == 0)
+def _bwd_partial(be, r, s, world, q, k, v, o, do, lse, scale, causal):
+    """Rank r's gradients for the chunk it holds at step s (None when the causal mask skips it)."""
+    kind = block_kind(r, source(r, s, world), causal)
+    return None if kind is None else be.bwd(q, k, v, o, do, lse, scale, kind == "diag")
+
+
+def _bwd_accumulate(be, st, s, part, dk_acc, dv_acc):
+    """Adds a step's partial gradients to dQ and to the held chunk's dK, dV accumulators."""
+    if part is None:
+        return
+    dq_p, dk_p, dv_p = part
+    be.accumulate(st.dq_acc, dq_p, st.first)
+    st.first = False
+    # the chunk's own rank starts its accumulators at step 0 (its diagonal block is never skipped)
+    be.accumulate(dk_acc, dk_p, s == 0)
+    be.accumulate(dv_acc, dv_p, s == 0)
 
 
 # ------------------------------------------------------------- distributed drivers
@@ -144,21 +151,31 @@ def ring_attention_bwd(q, k, v, o, do, lse, scale: float | None = None, causal: 
     st = _BwdState(be, q)
     kv = [k.contiguous(), v.contiguous()]
     acc = [be.f32_like(k), be.f32_like(v)]  # the held chunk's dK, dV accumulators
+    acc_reqs, nxt_acc = [], None
     for s in range(world):
         reqs, nxt_kv = [], None
         if s + 1 < world:  # the chunk itself moves on while this step computes
             nxt_kv = [torch.empty_like(t) for t in kv]
             reqs = _ring_exchange(kv, nxt_kv, rank, world, group)
-        _bwd_step(be, st, rank, s, world, q, kv[0], kv[1], o, do, lse, acc[0], acc[1], scale, causal)
-        if world > 1:  # its accumulators follow; after the last step this hands them back to the owner
-            nxt_acc = [torch.empty_like(t) for t in acc]
-            for req in _ring_exchange(acc, nxt_acc, rank, world, group):
-                req.wait()
+        # this step's gradients are computed while the held chunk's accumulators are still on their
+        # way from the previous holder; they are added once those have arrived
+        part = _bwd_partial(be, rank, s, world, q, kv[0], kv[1], o, do, lse, scale, causal)
+        for req in acc_reqs:
+            req.wait()
+        if nxt_acc is not None:
             acc = nxt_acc
+        _bwd_accumulate(be, st, s, part, acc[0], acc[1])
+        if world > 1:  # the accumulators follow their chunk; after the last step they reach the owner
+            nxt_acc = [torch.empty_like(t) for t in acc]
+            acc_reqs = _ring_exchange(acc, nxt_acc, rank, world, group)
         for req in reqs:
             req.wait()
         if nxt_kv is not None:
             kv = nxt_kv
+    for req in acc_reqs:
+        req.wait()
+    if nxt_acc is not None:
+        acc = nxt_acc
     return be.to_bf16(st.dq_acc), be.to_bf16(acc[0]), be.to_bf16(acc[1])
 
 
@@ -188,8 +205,8 @@ def ring_attention_bwd_emulated(qs, ks, vs, os_, dos, lses, scale: float | None 
     for s in range(world):
         for r in range(world):
             c = held[r]
-            _bwd_step(be, states[r], r, s, world, qs[r], c[0], c[1], os_[r], dos[r], lses[r], c[2], c[3], scale,
-                      causal)
+            part = _bwd_partial(be, r, s, world, qs[r], c[0], c[1], os_[r], dos[r], lses[r], scale, causal)
+            _bwd_accumulate(be, states[r], s, part, c[2], c[3])
         held = [held[(r - 1) % world] for r in range(world)]
     # after `world` rotations every chunk, with its accumulated dK and dV, is back at its owner
     return ([be.to_bf16(st.dq_acc) for st in states], [be.to_bf16(held[r][2]) for r in range(world)],
