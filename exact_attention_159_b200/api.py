@@ -37,6 +37,21 @@ def _need(t: torch.Tensor, name: str, dtype, shape):
     if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
         raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, got "
                          f"{t.dtype} {tuple(t.shape)} contiguous={t.is_contiguous()} cuda={t.is_cuda}")
+    _on_current_device(t, name)
+
+
+def _on_current_device(t: torch.Tensor, name: str):
+    # the library launches on the current device; a pointer into another GPU's memory must not reach it
+    if t.device.index is not None and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, but the current device is cuda:{torch.cuda.current_device()}")
+
+
+def _need_workspace(ws: torch.Tensor, nbytes: int):
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace: expected a contiguous CUDA tensor")
+    _on_current_device(ws, "workspace")
+    if ws.numel() * ws.element_size() < nbytes:
+        raise ValueError(f"workspace: {ws.numel() * ws.element_size()} bytes, {nbytes} needed")
 
 
 def fa_fwd(q, k, v, scale: float | None = None, causal: bool = False, out=None, lse=None, stream=None):
@@ -72,6 +87,7 @@ def fa_bwd(q, k, v, o, do, lse, scale: float | None = None, causal: bool = False
     ws_bytes = fa_bwd_workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace, ws_bytes)
     for t, nm in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
         _need(t, nm, _BF16, (B, H, N, d))
     check(_lib.lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
@@ -142,6 +158,7 @@ def fa_bwd_qk(q, k, v, o, do, lse, scale: float | None = None, causal: bool = Fa
     ws_bytes = fa_bwd_qk_workspace_size(B, Hq, Nq, d)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace, ws_bytes)
     _need(dq, "dq", _BF16, (B, Hq, Nq, d))
     for t, nm in ((dk, "dk"), (dv, "dv")):
         _need(t, nm, _BF16, (B, Hkv, Nk, d))
@@ -203,6 +220,7 @@ def fa_exp2_eval(x: torch.Tensor, mode: int = 0, stream=None) -> torch.Tensor:
     """2^x on the device: mode 0 = cubic software exp2, 1 = SFU ex2."""
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA float32 tensor")
+    _on_current_device(x, "x")
     y = torch.empty_like(x)
     check(_lib.lib().fa_exp2_eval(_ptr(x), _ptr(y), x.numel(), int(mode), _stream(stream)), "fa_exp2_eval")
     return y
@@ -224,6 +242,8 @@ def fa_sm_clock_probe(out: torch.Tensor | None = None, stream=None):
         out = torch.zeros(2, dtype=torch.int64, device="cuda")
     elif out.dtype != torch.int64 or not out.is_cuda or out.numel() != 2 or not out.is_contiguous():
         raise ValueError("out must be a contiguous CUDA int64 tensor of 2 elements")
+    else:
+        _on_current_device(out, "out")
     check(_lib.lib().fa_sm_clock_probe(_ptr(out), _stream(stream)), "fa_sm_clock_probe")
     if not own:
         return None

@@ -46,3 +46,9 @@ def test_diagnostic_helpers_refuse_cpu_buffers():
         api.fa_sm_clock_probe(torch.zeros(2, dtype=torch.int64))
     with pytest.raises(ValueError):
         api.fa_exp2_eval(torch.zeros(16, dtype=torch.float32))
+
+
+def test_workspace_must_be_a_device_buffer_of_the_needed_size():
+    from exact_attention_159_b200.api import _need_workspace
+    with pytest.raises(ValueError, match="CUDA"):
+        _need_workspace(torch.zeros(1 << 20, dtype=torch.uint8), 1024)   # host memory never reaches a kernel
