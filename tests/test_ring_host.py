@@ -151,3 +151,49 @@ def test_block_schedule():
             assert srcs[0] == r and sorted(srcs) == list(range(world))
     assert ring.block_kind(2, 1, True) == "full" and ring.block_kind(2, 2, True) == "diag"
     assert ring.block_kind(2, 3, True) is None and ring.block_kind(2, 3, False) == "full"
+
+
+def _group_worker(rank, world, port, out):
+    import torch.distributed as dist
+    from exact_attention_159_b200 import ring
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # two independent rings, ranks {0, 2} and {1, 3} (group ranks differ from global ranks)
+        groups = [dist.new_group([0, 2]), dist.new_group([1, 3])]
+        g = groups[rank % 2]
+        gr = dist.get_rank(g)
+        B, H, n, d = 1, 2, 8, 8
+        q, k, v, do = _inputs(B, H, 2 * n, d, seed=11 + rank % 2)  # each ring its own sequence
+        sl = slice(gr * n, (gr + 1) * n)
+        qc, kc, vc, doc = (t[:, :, sl].contiguous() for t in (q, k, v, do))
+        be = Fp64Backend()
+        o, lse = ring.ring_attention_fwd(qc, kc, vc, 0.4, True, group=g, backend=be)
+        dq, dk, dv = ring.ring_attention_bwd(qc, kc, vc, o, doc, lse, 0.4, True, group=g, backend=be)
+        out[rank] = [t.numpy() for t in (o, lse, dq, dk, dv)]
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_over_a_subgroup_of_ranks():
+    ctx = mp.get_context("spawn")
+    port = 29950 + (os.getpid() % 40)
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_group_worker, args=(4, port, out), nprocs=4, join=True, start_method="spawn")
+        res = dict(out)
+    B, H, n, d = 1, 2, 8, 8
+    for parity in (0, 1):
+        q, k, v, do = (t.numpy() for t in _inputs(B, H, 2 * n, d, seed=11 + parity))
+        for h in range(H):
+            o_ref, l_ref = OR.fwd(q[0, h], k[0, h], v[0, h], 0.4, True, nthreads=1)
+            dq_ref, dk_ref, dv_ref, _, _ = OR.bwd(q[0, h], k[0, h], v[0, h], do[0, h], 0.4, True, nthreads=1)
+            for gr, rank in enumerate((parity, parity + 2)):
+                sl = slice(gr * n, (gr + 1) * n)
+                o, lse, dq, dk, dv = res[rank]
+                np.testing.assert_allclose(o[0, h], o_ref[sl], atol=1e-12)
+                np.testing.assert_allclose(lse[0, h], l_ref[sl], atol=1e-12)
+                np.testing.assert_allclose(dq[0, h], dq_ref[sl], atol=1e-11)
+                np.testing.assert_allclose(dk[0, h], dk_ref[sl], atol=1e-11)
+                np.testing.assert_allclose(dv[0, h], dv_ref[sl], atol=1e-11)
