@@ -13,7 +13,11 @@ inside the timed region).  Multi-GPU (torchrun): every rank runs its own
 batch of heads (no collective on the data path), weak scaling.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
-bounded sample of the same workload on the host cores.
+bounded sample of the same job (forward and backward of one head) on the host
+cores.  The GPU line also carries `per_config`: forward and backward timings of
+every workload of the evaluation (the five configurations, the sweep's twelve
+runs included), and `cpu_baseline.per_config`: the oracle's wall time and
+GFLOPS on a bounded sample of each.
 """
 from __future__ import annotations
 
@@ -306,7 +310,7 @@ def run_gpu(args):
         prev_done[:] = ev_done
         prev_out[:] = ev_out
 
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = max(1, args.steps)
     e2e_step()
     stream.wait_stream(s_out)
     barrier()
@@ -346,8 +350,11 @@ def run_gpu(args):
                                 "fwd_of_measured_burst": round(100 * fwd_tf / pk["burst"], 2),
                                 "bwd_of_measured_burst": round(100 * bwd_tf / pk["burst"], 2)},
         "roofline": {"bound": "tensor", "kernel": f"{dominant} attention kernel", "achieved": round(ach, 2),
-                     "peak": pk["sustained"], "unit": "TFLOP/s", "frac": round(ach / pk["sustained"], 4),
-                     "peak_kind": f"{pk['source']} sustained bf16 (kernel timed inside a multi-second loop)",
+                     "peak": pk["burst"], "unit": "TFLOP/s", "frac": round(ach / pk["burst"], 4),
+                     "peak_kind": f"{pk['source']} burst bf16 GEMM (the timed region lasts "
+                                  f"{ms * 1e-3:.2f} s, well under a seconds-long sustained loop)",
+                     "frac_of_sustained": round(ach / pk["sustained"], 4),
+                     "fwd_frac": round(fwd_tf / pk["burst"], 4), "bwd_frac": round(bwd_tf / pk["burst"], 4),
                      "traffic": stored_traffic(dominant),
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)"},
         "e2e": {"value": round(job_tflops(f_fwd + f_bwd, world, e2e_ms), 2), "unit": "TFLOPS",
@@ -361,6 +368,9 @@ def run_gpu(args):
                                            f"the forward and the backward of the last {PROBE_KEEP} of {PROBE_STEPS} "
                                            f"untimed steps run back to back after the timed loop"},
     }
+    if not args.no_per_config:
+        # every rank times the same extra shapes; rank 0 reports its own numbers (untimed by the main loop)
+        result["per_config"] = gpu_per_config(api, reps=args.per_config_reps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     if world > 1:
@@ -370,52 +380,177 @@ def run_gpu(args):
         print(json.dumps(result), flush=True)
 
 
+# ------------------------------------------------------- per-config GPU timings
+def configurations():
+    """The evaluation's workloads, each with the passes its configuration names: (tag, workload id,
+    B, H, N, d, causal, stress, backward).  Workload 5 is the twelve-run backward sweep."""
+    from exact_attention_159_b200 import inputs as I
+    out = []
+    for wid, w in sorted(I.WORKLOADS.items()):
+        out.append((w["name"], wid, w["B"], w["H"], w["N"], w["d"], w["causal"], w["stress"], w["bwd"]))
+    for w in I.SWEEP:
+        out.append((w["name"], 5, w["B"], w["H"], w["N"], w["d"], w["causal"], w["stress"], True))
+    return out
+
+
+def device_inputs(seed, B, H, N, d, stress, with_do):
+    """Seeded N(0, 1) bf16 inputs drawn on the device with torch's generator (timing only: the same
+    distributions and the same rescale-stress construction as the host generator, not its bits)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    shape = (B, H, N, d)
+    t = {k: torch.randn(shape, generator=g, device="cuda", dtype=torch.float32) for k in ("q", "k", "v")}
+    if stress:
+        u = torch.randn(d, generator=g, device="cuda", dtype=torch.float64)
+        u = (u / u.norm()).float()
+        for k in ("q", "k"):
+            a = torch.rand((B, H, N, 1), generator=g, device="cuda", dtype=torch.float32) * 8.0
+            t[k] += a * u
+    if with_do:
+        t["do"] = torch.randn(shape, generator=g, device="cuda", dtype=torch.float32)
+    return {k: v.to(torch.bfloat16) for k, v in t.items()}
+
+
+def gpu_per_config(api, reps=5):
+    """Forward and backward device time of every workload: `reps` calls each, the L2 flushed
+    (a 256 MB write) before every timed call, CUDA events on the launching stream; medians."""
+    import torch
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rows = []
+    for tag, wid, B, H, N, d, causal, stress, bwd in configurations():
+        x = device_inputs(1000 * wid + 7, B, H, N, d, stress, bwd)
+        scale = 1.0 / math.sqrt(d)
+        o, lse = api.fa_fwd(x["q"], x["k"], x["v"], scale, causal)
+        f_fwd, f_bwd = flops(B, H, N, d, causal)
+        ws = torch.empty(api.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda") if bwd else None
+        grads = [torch.empty_like(x["q"]) for _ in range(3)] if bwd else None
+
+        def timed(fn, prof_which=None):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.zero_()
+            if prof_which is not None:
+                api.fa_profile_next(prof_which, ev[2], ev[3])
+            ev[0].record(stream)
+            fn()
+            ev[1].record(stream)
+            return ev
+
+        def fwd_call():
+            api.fa_fwd(x["q"], x["k"], x["v"], scale, causal, out=o, lse=lse)
+
+        def bwd_call():
+            api.fa_bwd(x["q"], x["k"], x["v"], o, x["do"], lse, scale, causal, dq=grads[0], dk=grads[1],
+                       dv=grads[2], workspace=ws)
+
+        fwd_call()
+        if bwd:
+            bwd_call()
+        fe = [timed(fwd_call) for _ in range(reps)]
+        be = [timed(bwd_call, 1) for _ in range(reps)] if bwd else []
+        torch.cuda.synchronize()
+        rc, detail = api.fa_last_device_status()
+        if rc != 0:
+            raise RuntimeError(f"device status {rc} ({detail:#x}) in the per-config timings ({tag})")
+        f_ms = statistics.median(e[0].elapsed_time(e[1]) for e in fe)
+        row = {"config": tag, "workload": wid, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+               "fwd_ms": round(f_ms, 4), "fwd_tflops": round(f_fwd / (f_ms * 1e-3) / 1e12, 2)}
+        if bwd:
+            b_ms = statistics.median(e[0].elapsed_time(e[1]) for e in be)
+            m_ms = statistics.median(e[2].elapsed_time(e[3]) for e in be)
+            row.update(bwd_ms=round(b_ms, 4), bwd_tflops=round(f_bwd / (b_ms * 1e-3) / 1e12, 2),
+                       bwd_main_ms=round(m_ms, 4), bwd_main_tflops=round(f_bwd / (m_ms * 1e-3) / 1e12, 2))
+        rows.append(row)
+        del x, o, lse, ws, grads
+    return {"rows": rows, "inputs": "seeded N(0,1) bf16 drawn on the device (torch generator), stress "
+                                    "construction for workload 3", "timing": f"median of {reps} calls, L2 flushed "
+                                    "before each, CUDA events; bwd = the whole fa_bwd call (3 kernels), bwd_main "
+                                    "= its main kernel", "flops": "fwd 4*B*H*N^2*d, bwd 2.5x, halved for causal"}
+
+
 # ---------------------------------------------------------------- CPU oracle
-def _oracle_sample(budget_s):
-    """Oracle forward on query rows of head (0, 0) of the workload, every `stride`-th row,
-    stride chosen so the sample is ~budget_s of work on this host."""
+def _visible_rows(N, causal):
+    """Number of keys each query row sees (square problems)."""
+    import numpy as np
+    return np.arange(1, N + 1, dtype=np.float64) if causal else np.full(N, float(N))
+
+
+def oracle_head(wid, B, H, N, d, stress, bwd):
+    """fp64 operands of head (0, 0) of a workload (exact widenings of the seeded bf16 inputs)."""
+    from exact_attention_159_b200 import inputs as I
+    bits = I.head_inputs(wid, B, H, N, d, 0, 0, stress=stress, with_do=bwd)
+    return {k: I.bf16_bits_to_f64(v) for k, v in bits.items()}
+
+
+def oracle_sample(wid, B, H, N, d, causal, stress, bwd, fwd_budget_s, threads, n_bwd_rows=64, x=None):
+    """The fp64 oracle on head (0, 0) of one workload: forward of every stride-th query row (stride
+    chosen for ~fwd_budget_s), and, with bwd, the backward for 64 sampled query rows (dQ) and 64
+    sampled key rows (dK, dV).  FLOPs are those of the outputs produced, each GEMM counted once:
+    forward 4*d per visible (query, key) pair; backward 4*d per visible pair over every row (S and dP,
+    which LSE and D need) + 2*d per visible pair of the dQ rows + 4*d per visible pair of the dK / dV
+    rows (at full size these add up to the 10*d per pair, 2.5x the forward, of the convention)."""
     import numpy as np
 
-    from exact_attention_159_b200 import inputs as I
     from oracle import oracle as OR
 
-    w = WORKLOAD
-    N, d = w["N"], w["d"]
-    seed = w["seed_workload"]
-    # head (0, 0) is the first N*d draws of each tensor's stream
-    q, k, v = (I.bf16_bits_to_f64(I.normal_bf16(I.seed_for(seed, t), (N, d))) for t in ("q", "k", "v"))
-    threads = OR.default_threads()
-    # calibrate on a small row set
-    probe = np.arange(0, N, 512)
+    if x is None:
+        x = oracle_head(wid, B, H, N, d, stress, bwd)
+    scale = 1.0 / math.sqrt(d)
+    vis = _visible_rows(N, causal)
+    probe = np.arange(0, N, max(1, N // 64))
     t = time.perf_counter()
-    OR.fwd(q, k, v, 1.0 / math.sqrt(d), w["causal"], rows=probe, nthreads=threads)
-    dt = max(time.perf_counter() - t, 1e-3)
-    stride = max(1, int(512 * dt / budget_s))
+    OR.fwd(x["q"], x["k"], x["v"], scale, causal, rows=probe, nthreads=threads)
+    per_row = max(time.perf_counter() - t, 1e-4) / probe.size
+    stride = max(1, int(math.ceil(N * per_row / fwd_budget_s)))
     rows = np.arange(stride // 2, N, stride)
-    return q, k, v, rows, stride, threads
+    t = time.perf_counter()
+    OR.fwd(x["q"], x["k"], x["v"], scale, causal, rows=rows, nthreads=threads)
+    f_s = time.perf_counter() - t
+    f_fl = float(4.0 * d * vis[rows].sum())
+    out = {"fwd": {"seconds": round(f_s, 3), "gflops": round(f_fl / f_s / 1e9, 3), "flops": f_fl,
+                   "sample": f"{rows.size} of {N} query rows (every {stride}th) of head (0,0)"}}
+    if bwd:
+        rng = np.random.default_rng(wid * 100 + N + d + int(causal))
+        qr = np.unique(np.concatenate([[0, N - 1], rng.choice(N, size=min(N, n_bwd_rows), replace=False)]))
+        kr = np.unique(np.concatenate([[0, N - 1], rng.choice(N, size=min(N, n_bwd_rows), replace=False)]))
+        t = time.perf_counter()
+        OR.bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, qrows=qr, krows=kr, nthreads=threads)
+        b_s = time.perf_counter() - t
+        kvis = (N - kr).astype(np.float64) if causal else np.full(kr.size, float(N))
+        b_fl = float(4.0 * d * vis.sum() + 2.0 * d * vis[qr].sum() + 4.0 * d * kvis.sum())
+        out["bwd"] = {"seconds": round(b_s, 3), "gflops": round(b_fl / b_s / 1e9, 3), "flops": b_fl,
+                      "sample": f"head (0,0): LSE and D of all {N} rows, dQ of {qr.size} query rows, "
+                                f"dK and dV of {kr.size} key rows"}
+    return out
 
 
 def cpu_baseline(budget_s=15.0):
-    import numpy as np
-
+    """The oracle on every workload (head (0, 0), bounded samples); the headline value is the bench
+    workload's forward + backward sample."""
     from oracle import oracle as OR
 
-    q, k, v, rows, stride, threads = _oracle_sample(budget_s)
-    w = WORKLOAD
-    t = time.perf_counter()
-    OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
-    dt = time.perf_counter() - t
-    vis = (rows + 1) if w["causal"] else np.full(rows.shape, w["N"])
-    fl = float(4.0 * w["d"] * vis.sum())
-    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
-            "sample": f"fp64 oracle forward of {rows.size} query rows (every {stride}th) of head (0,0) of the "
-                      f"workload, {dt:.1f} s; FLOPs counted as 4*d per visible key",
-            "seconds": round(dt, 2)}
+    threads = OR.default_threads()
+    per = []
+    head = None
+    t0 = time.perf_counter()
+    for tag, wid, B, H, N, d, causal, stress, bwd in configurations():
+        fwd_budget = budget_s / 10.0 if wid == 4 else budget_s / 40.0
+        r = oracle_sample(wid, B, H, N, d, causal, stress, bwd, fwd_budget, threads)
+        row = {"config": tag, "workload": wid, "B": B, "H": H, "N": N, "d": d, "causal": causal, **r}
+        per.append(row)
+        if wid == 4:
+            head = r
+    fl = head["fwd"]["flops"] + head["bwd"]["flops"]
+    sec = head["fwd"]["seconds"] + head["bwd"]["seconds"]
+    return {"value": round(fl / sec / 1e12, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
+            "sample": "fp64 oracle, head (0,0) of the bench workload: forward of "
+                      f"{head['fwd']['sample'].split(' (')[0]}, and the backward ({head['bwd']['sample']}); "
+                      "FLOPs of the outputs produced, each GEMM counted once",
+            "seconds": round(sec, 2), "per_config": per, "per_config_seconds": round(time.perf_counter() - t0, 1)}
 
 
 def run_reference(args):
-    import numpy as np
-
     from oracle import oracle as OR
 
     rank = int(os.environ.get("RANK", "0"))
@@ -423,24 +558,25 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOAD
-    per_step = max(0.5, min(6.0, 150.0 / max(1, args.steps + args.warmup)))
-    q, k, v, rows, stride, threads = _oracle_sample(per_step)
-    vis = (rows + 1) if w["causal"] else np.full(rows.shape, w["N"])
-    fl = float(4.0 * w["d"] * vis.sum())
-    for _ in range(args.warmup):
-        OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        OR.fwd(q, k, v, 1.0 / math.sqrt(w["d"]), w["causal"], rows=rows, nthreads=threads)
-    dt = (time.perf_counter() - t) / max(1, args.steps)
-    value = fl / dt / 1e12
-    sample = (f"fp64 oracle forward of {rows.size} query rows (every {stride}th) of head (0,0) per step; "
-              f"FLOPs counted as 4*d per visible key")
+    threads = OR.default_threads()
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    fwd_budget = max(0.2, min(1.0, 30.0 / max(1, args.steps + args.warmup)))
+    x = oracle_head(w["seed_workload"], B, H, N, d, False, True)
+    samples = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w["seed_workload"], B, H, N, d, causal, False, True, fwd_budget, threads, x=x)
+        if i >= args.warmup:
+            samples.append(r)
+    fl = sum(r["fwd"]["flops"] + r["bwd"]["flops"] for r in samples)
+    sec = sum(r["fwd"]["seconds"] + r["bwd"]["seconds"] for r in samples)
+    value = fl / sec / 1e12
+    sample = (f"fp64 oracle per step, head (0,0) of the workload: forward of {samples[0]['fwd']['sample'].split(' (')[0]}"
+              f" and the backward ({samples[0]['bwd']['sample']}); FLOPs of the outputs produced, each GEMM counted once")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
-        "config": config_dict(world),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec / max(1, args.steps) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16)", "config": config_dict(world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -483,6 +619,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-configuration GPU timings")
+    ap.add_argument("--per-config-reps", type=int, default=5, help="timed calls per configuration")
     ap.add_argument("--profile", choices=["fwd", "bwd"], help="plain calls on --shape for ncu captures")
     ap.add_argument("--shape", default="1,16,16384,128", help="B,H,N,d for --profile")
     ap.add_argument("--causal", type=int, default=1, help="causal flag for --profile")

@@ -204,7 +204,8 @@ def fa_last_device_status(stream=None) -> tuple[int, int]:
     return int(rc), int(detail.value)
 
 
-def fa_set_softmax_options(tau: float = 8.0, poly: int = 0) -> None:
+def fa_set_softmax_options(tau: float = 8.0, poly: int = -1) -> None:
+    """Rescale threshold and cubic-exp2 share (pairs per 16; -1 = per-head-dim default)."""
     check(_lib.lib().fa_set_softmax_options(float(tau), int(poly)), "fa_set_softmax_options")
 
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -20,7 +21,9 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kPoly16 = 4;     // exponentials per 16 evaluated by the cubic when the polynomial path is on
+// Forward: element pairs out of every 16 whose exponentials take the FMA-pipe cubic by default,
+// per head dimension (index 0: d = 64, 1: d = 128).
+constexpr int kPolyDefault[2] = {0, 0};
 constexpr int kBwdPoly16 = 0;  // backward: the SFU alone measured faster than any polynomial share
 
 __device__ int g_status;  // first device-side failure (wait site), 0 = none
@@ -32,11 +35,15 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
-float g_tau = fa::kRescaleTau;
-int g_poly = 0;  // forward default: SFU only (measured faster on B200 than the 1/4 polynomial share)
-int g_fwd_pair = 0;  // 1: forward at d = 128 on cluster pairs (cta_group::2 UMMA)
-int g_bwd_pair = 0;  // 1: backward at d = 128 on cluster pairs (cta_group::2 UMMA)
-cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};  // one-shot [fwd|bwd][start|stop]
+// Process-wide switches (atomics: a setter racing with calls on other threads is not a data race;
+// which setting a concurrent call sees is unspecified).
+std::atomic<float> g_tau{fa::kRescaleTau};
+std::atomic<int> g_poly{-1};      // cubic pairs per 16 in the forward; -1 = kPolyDefault for the head dimension
+std::atomic<int> g_fwd_pair{0};   // 1: forward at d = 128 on cluster pairs (cta_group::2 UMMA)
+std::atomic<int> g_bwd_pair{0};   // 1: backward at d = 128 on cluster pairs (cta_group::2 UMMA)
+// One-shot profiling events [fwd|bwd][start|stop], per host thread: armed by fa_profile_next and
+// consumed by the next fa_fwd* / fa_bwd* call made on the same thread.
+thread_local cudaEvent_t g_prof[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
 
 // Records the pending start event of `which` (if any) on `st`; returns whether one was pending.
 bool prof_begin(int which, cudaStream_t st) {
@@ -167,6 +174,29 @@ int launch_fwd2(const CUtensorMap& q, const CUtensorMap& k64, const CUtensorMap&
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// The forward with `poly` (0, 1, 2 or 4) of every 16 element pairs on the cubic.
+template <int D, bool C>
+int launch_fwd_poly(int poly, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                    const fa::FwdParams& prm, cudaStream_t st) {
+  switch (poly) {
+    case 0: return launch_fwd<D, C, 0>(q, k, v, prm, st);
+    case 1: return launch_fwd<D, C, 1>(q, k, v, prm, st);
+    case 2: return launch_fwd<D, C, 2>(q, k, v, prm, st);
+    default: return launch_fwd<D, C, 4>(q, k, v, prm, st);
+  }
+}
+
+template <bool C>
+int launch_fwd2_poly(int poly, const CUtensorMap& q, const CUtensorMap& k64, const CUtensorMap& v,
+                     const fa::Fwd2Params& prm, cudaStream_t st) {
+  switch (poly) {
+    case 0: return launch_fwd2<C, 0>(q, k64, v, prm, st);
+    case 1: return launch_fwd2<C, 1>(q, k64, v, prm, st);
+    case 2: return launch_fwd2<C, 2>(q, k64, v, prm, st);
+    default: return launch_fwd2<C, 4>(q, k64, v, prm, st);
+  }
+}
+
 template <int D, bool C>
 int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
                const CUtensorMap& dq_acc, const fa::BwdParams& prm, cudaStream_t st) {
@@ -262,7 +292,8 @@ const char* fa_strerror(int status) {
 }
 
 int fa_set_softmax_options(float tau, int poly) {
-  if (!(tau >= 0.0f && tau <= 16.0f) || (poly != 0 && poly != 1)) return FA_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f && tau <= 16.0f) || (poly != -1 && poly != 0 && poly != 1 && poly != 2 && poly != 4))
+    return FA_ERR_INVALID_ARG;
   g_tau = tau;
   g_poly = poly;
   return FA_OK;
@@ -302,11 +333,12 @@ int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, 
   const int tiles = (Nq + 127) / 128;
   prm.n_pairs = (tiles + 1) / 2;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.tau = g_tau;
+  prm.tau = g_tau.load(std::memory_order_relaxed);
   prm.status = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool poly = g_poly != 0;
-  if (d == 128 && g_fwd_pair && Hq == Hkv && Nq == Nk) {
+  const int poly_set = g_poly.load(std::memory_order_relaxed);
+  const int poly = poly_set >= 0 ? poly_set : kPolyDefault[d == 128 ? 1 : 0];
+  if (d == 128 && g_fwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
     CUtensorMap mk64;
     if (!make_map(&mk64, K, BH, Nk, d, 64)) return FA_ERR_CUDA;
     fa::Fwd2Params p2;
@@ -319,25 +351,17 @@ int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, 
     p2.tau = prm.tau;
     p2.status = prm.status;
     const bool prof2 = prof_begin(0, st);
-    if (causal)
-      rc = poly ? launch_fwd2<true, kPoly16>(mq, mk64, mv, p2, st) : launch_fwd2<true, 0>(mq, mk64, mv, p2, st);
-    else
-      rc = poly ? launch_fwd2<false, kPoly16>(mq, mk64, mv, p2, st) : launch_fwd2<false, 0>(mq, mk64, mv, p2, st);
+    rc = causal ? launch_fwd2_poly<true>(poly, mq, mk64, mv, p2, st) : launch_fwd2_poly<false>(poly, mq, mk64, mv, p2, st);
     if (prof2) prof_end(0, st);
     return rc;
   }
   const bool prof = prof_begin(0, st);
-  if (d == 128) {
-    if (causal)
-      rc = poly ? launch_fwd<128, true, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<128, true, 0>(mq, mk, mv, prm, st);
-    else
-      rc = poly ? launch_fwd<128, false, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<128, false, 0>(mq, mk, mv, prm, st);
-  } else {
-    if (causal)
-      rc = poly ? launch_fwd<64, true, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<64, true, 0>(mq, mk, mv, prm, st);
-    else
-      rc = poly ? launch_fwd<64, false, kPoly16>(mq, mk, mv, prm, st) : launch_fwd<64, false, 0>(mq, mk, mv, prm, st);
-  }
+  if (d == 128)
+    rc = causal ? launch_fwd_poly<128, true>(poly, mq, mk, mv, prm, st)
+                : launch_fwd_poly<128, false>(poly, mq, mk, mv, prm, st);
+  else
+    rc = causal ? launch_fwd_poly<64, true>(poly, mq, mk, mv, prm, st)
+                : launch_fwd_poly<64, false>(poly, mq, mk, mv, prm, st);
   if (prof) prof_end(0, st);
   return rc;
 }
@@ -428,7 +452,7 @@ int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const 
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   const bool prof = prof_begin(1, st);
-  if (d == 128 && g_bwd_pair && Hq == Hkv && Nq == Nk) {
+  if (d == 128 && g_bwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
     CUtensorMap mq64, mdo64, macc64;
     if (!make_map(&mq64, Q, BH, Nq, d, 64) || !make_map(&mdo64, dO, BH, Nq, d, 64) ||
         !make_acc_map(&macc64, dq_acc, BH, npad, d, 64))

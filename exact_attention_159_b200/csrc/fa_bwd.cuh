@@ -1,8 +1,9 @@
 // fa_bwd.cuh -- backward exact attention on sm_100a.
 //
 // P is recomputed from the saved log-sum-exp instead of being stored
-// (FlashAttention-4 pages: backward pass with intermediates kept in TMEM,
-// "using TMEM to store backward intermediates instead of SMEM").  Three
+// ("NVIDIA Blackwell: FlashAttention-4 Overcomes Memory Bottlenecks": the
+// backward keeps its intermediates in tensor memory rather than shared
+// memory, which cuts shared-memory traffic).  Three
 // kernels run on the caller's stream:
 //   bwd_prep_kernel    D_i = dO_i . O_i, LSE2_i = LSE_i * log2(e) (+inf on the
 //                      padding rows of the last tile), dQ_acc = 0

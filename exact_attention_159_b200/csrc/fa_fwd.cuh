@@ -23,14 +23,15 @@
 //   column) is written back over the first 64 columns of S_t and read from
 //   there by the P.V MMA; O_t fp32, D columns at 256 + D*t.
 // Online softmax in base 2 with the running row maximum m (log2 units) and
-// conditional rescaling ("adaptive online softmax rescaling ... only when
-// maximum values change significantly"): O and l are rescaled only when the
+// conditional rescaling (ainvest page, "The Technical Edge": the running
+// output is rescaled only when the row maximum has moved by a large amount):
+// O and l are rescaled only when the
 // tile maximum exceeds the reference maximum by more than tau = 8; otherwise
 // the stale reference is kept, so P <= 2^8.  The result is exact either way
 // because O / l and LSE use the same reference.
-// A fixed share of the exponentials of interior tiles runs as the cubic
-// polynomial on the FMA pipe, the rest on the SFU ("cubic polynomials ...
-// reduces SFU contention").
+// A fixed share (POLY16 / 16) of the exponentials of interior tiles runs as the cubic
+// polynomial on the FMA pipe, the rest on the SFU (same section: a cubic on
+// the CUDA cores takes load off the special-function units).
 #pragma once
 
 #include <type_traits>
@@ -320,6 +321,8 @@ __global__ void __launch_bounds__(640, 1)
       float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
       // The two paths are separate code, so the tiles that use the cubic for part of their
       // exponentials issue no SFU operation for that part (a select between the two would).
+      // POLY16 of every 16 element pairs (evenly spaced) take the cubic
+      constexpr int kPolyStride = POLY16 > 0 ? 16 / POLY16 : 16;
       auto exp_store = [&](auto poly_tag) {
         constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(640, 1)
             const int c = 32 * cc + 2 * e;
             const float2 x = __ffma2_rn(make_float2(S(c), S(c + 1)), c2, nm2);
             float2 p;
-            if (kPoly && (e & 7) < POLY16 / 2) {
+            if (kPoly && e % kPolyStride == 0) {
               p = exp2_poly2(x);
             } else {
               p.x = exp2_sfu(x.x);

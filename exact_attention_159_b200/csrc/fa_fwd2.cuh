@@ -276,7 +276,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
           const int c = 32 * cc + 2 * e;
           const float2 x = __ffma2_rn(make_float2(S(c), S(c + 1)), c2, nm2);
           float2 p;
-          if (!edge && (e & 7) < POLY16 / 2) {
+          if (!edge && POLY16 > 0 && e % (POLY16 > 0 ? 16 / POLY16 : 16) == 0) {
             p = exp2_poly2(x);
           } else {
             p.x = exp2_sfu(x.x);

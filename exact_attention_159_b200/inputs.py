@@ -49,13 +49,16 @@ def uniform(seed: int, start: int, count: int) -> np.ndarray:
     return (z >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
 
 
-def normal(seed: int, count: int) -> np.ndarray:
-    """``count`` fp64 standard normals of stream ``seed`` (Box-Muller, fp64)."""
+def normal(seed: int, count: int, start: int = 0) -> np.ndarray:
+    """``count`` fp64 standard normals of stream ``seed`` (Box-Muller, fp64), starting at normal
+    number ``start`` of the stream (even, so that Box-Muller pairs stay aligned)."""
+    if start % 2:
+        raise ValueError("start must be even")
     out = np.empty(count, dtype=np.float64)
     pairs = (count + 1) // 2
     for p0 in range(0, pairs, _CHUNK):
         p1 = min(pairs, p0 + _CHUNK)
-        u = uniform(seed, 2 * p0, 2 * (p1 - p0)).reshape(-1, 2)
+        u = uniform(seed, start + 2 * p0, 2 * (p1 - p0)).reshape(-1, 2)
         r = np.sqrt(-2.0 * np.log1p(-u[:, 0]))  # 1 - u in (0, 1]
         t = 2.0 * np.pi * u[:, 1]
         z = np.stack([r * np.cos(t), r * np.sin(t)], axis=1).reshape(-1)
@@ -110,6 +113,30 @@ def attention_inputs(workload: int, B: int, H: int, N: int, d: int, *,
     out["v"] = normal_bf16(seed_for(workload, "v"), shape)
     if with_do:
         out["do"] = normal_bf16(seed_for(workload, "do"), shape)
+    return out
+
+
+def head_inputs(workload: int, B: int, H: int, N: int, d: int, b: int, h: int, *,
+                stress: bool = False, with_do: bool = False) -> dict:
+    """The (b, h) slice (N x d bf16 bit arrays) of ``attention_inputs(workload, B, H, N, d, ...)``,
+    drawn on its own from the counter-based streams (equal to slicing the full tensors)."""
+    row0 = (b * H + h) * N  # first row of this head in the B*H*N rows of each tensor
+    out = {}
+    if stress:
+        u = normal(seed_for(workload, "u"), d)
+        u /= np.sqrt(np.sum(u * u))
+        rows = B * H * N
+        for name, first in (("q", row0), ("k", rows + row0)):
+            a = uniform(seed_for(workload, "offsets"), first, N) * 8.0
+            x = normal(seed_for(workload, name), N * d, start=row0 * d).reshape(N, d)
+            x += a[:, None] * u[None, :]
+            out[name] = f64_to_bf16_bits(x)
+    else:
+        for name in ("q", "k"):
+            out[name] = f64_to_bf16_bits(normal(seed_for(workload, name), N * d, start=row0 * d)).reshape(N, d)
+    names = ("v", "do") if with_do else ("v",)
+    for name in names:
+        out[name] = f64_to_bf16_bits(normal(seed_for(workload, name), N * d, start=row0 * d)).reshape(N, d)
     return out
 
 

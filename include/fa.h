@@ -163,9 +163,16 @@ int fa_last_device_status(void* stream, int* detail);
 /*
  * Tuning of the forward softmax (process-wide; for A/B comparisons).
  * tau: rescale threshold in log2 units (0 <= tau <= 16; 0 = rescale whenever
- * the running maximum grows; default 8).  poly: 1 = evaluate a quarter of the
- * exponentials of interior tiles with the FMA-pipe cubic, 0 = all on the SFU
- * (default 0).  Returns FA_ERR_INVALID_ARG for values out of range.
+ * the running maximum grows; default 8).  poly: how many of every 16 element
+ * pairs of an interior tile take the FMA-pipe cubic exp2 instead of the SFU:
+ * 0 (all on the SFU), 1, 2 or 4 (a sixteenth, an eighth, a quarter); -1
+ * restores the library's default for each head dimension.  Returns
+ * FA_ERR_INVALID_ARG for values out of range.
+ *
+ * This and the two variant setters below change process-wide settings.  They
+ * are safe to call from any thread, but a call of fa_fwd* / fa_bwd* running
+ * at the same time on another thread may see the old or the new setting: set
+ * them between calls.
  */
 int fa_set_softmax_options(float tau, int poly);
 
@@ -203,11 +210,13 @@ int fa_exp2_eval(const float* x, float* y, int64_t n, int mode, void* stream);
 
 /*
  * Profiling hook (used by the benchmark to time one kernel inside a call):
- * when start_event and stop_event are cudaEvent_t handles, the NEXT fa_fwd
- * (which = 0) or fa_bwd (which = 1) call records start_event on its stream
- * immediately before its main attention kernel and stop_event immediately
- * after it, then forgets both.  NULL, NULL clears a pending request.
- * Returns FA_ERR_INVALID_ARG for another `which` or a half-NULL pair.
+ * when start_event and stop_event are cudaEvent_t handles, the NEXT fa_fwd*
+ * (which = 0) or fa_bwd* (which = 1) call made on the SAME host thread
+ * records start_event on its stream immediately before its main attention
+ * kernel and stop_event immediately after it, then forgets both.  Requests
+ * are per thread, so calls on other threads neither see nor consume them.
+ * NULL, NULL clears a pending request.  Returns FA_ERR_INVALID_ARG for
+ * another `which` or a half-NULL pair.
  */
 int fa_profile_next(int which, void* start_event, void* stop_event);
 

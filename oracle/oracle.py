@@ -128,28 +128,6 @@ def bwd(q, k, v, do, scale: float, causal: bool, qrows=None, krows=None,
     return dq, dk, dv, lse, dsum
 
 
-def fwd_all(Q, K, V, scale: float, causal: bool, nthreads: int | None = None):
-    """Forward over a whole B x H x N x d batch (fp64 arrays): returns O, LSE."""
-    B, H, N, d = Q.shape
-    O = np.zeros((B, H, N, d)); L = np.zeros((B, H, N))
-    for b in range(B):
-        for h in range(H):
-            O[b, h], L[b, h] = fwd(Q[b, h], K[b, h], V[b, h], scale, causal, nthreads=nthreads)
-    return O, L
-
-
-def bwd_all(Q, K, V, dO, scale: float, causal: bool, nthreads: int | None = None):
-    """Backward over a whole B x H x N x d batch: returns dQ, dK, dV, LSE, D."""
-    B, H, N, d = Q.shape
-    dQ = np.zeros((B, H, N, d)); dK = np.zeros_like(dQ); dV = np.zeros_like(dQ)
-    L = np.zeros((B, H, N)); Dd = np.zeros((B, H, N))
-    for b in range(B):
-        for h in range(H):
-            dQ[b, h], dK[b, h], dV[b, h], L[b, h], Dd[b, h] = bwd(Q[b, h], K[b, h], V[b, h], dO[b, h],
-                                                                  scale, causal, nthreads=nthreads)
-    return dQ, dK, dV, L, Dd
-
-
 def gqa_fwd(Q, K, V, scale: float, causal: bool, rows=None, nthreads: int | None = None, lib=None):
     """Forward of one batch entry with Hq query heads over Hkv = Hq / G key/value heads
     (``Q``: Hq x nq x d, ``K``/``V``: Hkv x nk x d): query head h reads key/value head h // G."""

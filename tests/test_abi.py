@@ -112,9 +112,13 @@ def test_workspace_size(lib):
 
 def test_softmax_options_validation(lib):
     assert lib.fa_set_softmax_options(-1.0, 1) == _lib.FA_ERR_INVALID_ARG
-    assert lib.fa_set_softmax_options(8.0, 2) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_set_softmax_options(8.0, 3) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_set_softmax_options(8.0, 8) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_set_softmax_options(8.0, -2) == _lib.FA_ERR_INVALID_ARG
+    for share in (-1, 1, 2, 4):
+        assert lib.fa_set_softmax_options(8.0, share) == _lib.FA_OK
     assert lib.fa_set_softmax_options(0.0, 0) == _lib.FA_OK
-    assert lib.fa_set_softmax_options(8.0, 1) == _lib.FA_OK
+    assert lib.fa_set_softmax_options(8.0, -1) == _lib.FA_OK
 
 
 def test_exp2_eval_validation(lib):

@@ -21,7 +21,7 @@ def _device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     build.build()
-    api.fa_set_softmax_options(8.0, 0)
+    api.fa_set_softmax_options(8.0, -1)
     yield
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == (0, 0)
@@ -43,12 +43,16 @@ def check_fwd(case, o, lse, heads, rows_per_head, label):
     return worst_o, worst_l
 
 
-def check_bwd(case, grads, heads, nq, nk, label):
+def check_bwd(case, grads, heads, nq, nk, label, extra_k=None):
+    """Relative L2 of dQ / dK / dV against the oracle on sampled rows of `heads` (all rows when
+    nq / nk is None); `extra_k` adds key rows to every head's sample (e.g. whole key tiles)."""
     dQ, dK, dV = (bf16_to_f64(g) for g in grads)
     worst = {"dQ": 0.0, "dK": 0.0, "dV": 0.0}
     for (b, h) in heads:
         qr = None if nq is None else sample_rows(case.N, nq, 31 * b + h)
         kr = None if nk is None else sample_rows(case.N, nk, 37 * b + h + 1)
+        if kr is not None and extra_k is not None:
+            kr = np.unique(np.concatenate([kr, np.asarray(extra_k, dtype=np.int64)]))
         dq, dk, dv, _, _ = case.oracle_bwd(b, h, qr, kr)
         qs = np.arange(case.N) if qr is None else qr
         ks = np.arange(case.N) if kr is None else kr
@@ -90,7 +94,10 @@ def test_long_context_forward_backward_32768():
     o, lse = c.fwd_gpu()
     check_fwd(c, o, lse, all_heads(c), 48, "fwd causal B1 H16 N32768")
     grads = c.bwd_gpu(o, lse)
-    check_bwd(c, grads, [(0, 5)], 64, 64, "bwd causal B1 H16 N32768")
+    # heads 0, 7 and 15 run in different waves of the heaviest-first CTA order; the first and the
+    # last key tile (rows 0..127 and N-128..N-1) are checked in full on each
+    edge_keys = np.concatenate([np.arange(128), np.arange(c.N - 128, c.N)])
+    check_bwd(c, grads, [(0, 0), (0, 7), (0, 15)], 64, 64, "bwd causal B1 H16 N32768", extra_k=edge_keys)
     # invariants over every head: sum_j dV_j = sum_i dO_i, sum_j dK_j = 0
     dK = bf16_to_f64(grads[1])
     dV = bf16_to_f64(grads[2])
@@ -111,9 +118,10 @@ SWEEP = [(B, N, d, causal) for (B, N) in ((8, 2048), (2, 8192), (1, 16384)) for 
 def test_backward_sweep(B, N, d, causal):
     c = Case(B, 16, N, d, causal, seed_workload=5, bwd=True)
     o, lse = c.fwd_gpu()
-    heads = [(B - 1, 7)]
+    heads = [(0, 0), (B - 1, 7)]
     check_fwd(c, o, lse, heads, 48, f"sweep fwd B{B} N{N} d{d} causal={causal}")
-    check_bwd(c, c.bwd_gpu(o, lse), heads, 48, 48, f"sweep bwd B{B} N{N} d{d} causal={causal}")
+    check_bwd(c, c.bwd_gpu(o, lse), heads, 48, 48, f"sweep bwd B{B} N{N} d{d} causal={causal}",
+              extra_k=np.arange(N - 128, N))
 
 
 # --------------------------------------------------------------- edge cases
@@ -137,16 +145,17 @@ def test_several_tiles_and_heads_full(d, causal):
     check_bwd(c, c.bwd_gpu(o, lse), all_heads(c), None, None, f"multi bwd d{d} c{int(causal)}")
 
 
-@pytest.mark.parametrize("tau,poly", [(8.0, 1), (0.0, 0), (0.0, 1), (8.0, 0)])
-def test_rescale_and_exp_variants_agree(tau, poly):
-    c = Case(1, 4, 2048, 128, False, seed_workload=3, stress=True)
-    api.fa_set_softmax_options(8.0, 0)
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("tau,poly", [(8.0, 4), (8.0, 2), (8.0, 1), (0.0, 0), (0.0, 4), (8.0, 0)])
+def test_rescale_and_exp_variants_agree(tau, poly, d):
+    c = Case(1, 4, 2048, d, False, seed_workload=3, stress=True)
+    api.fa_set_softmax_options(8.0, -1)
     o_ref_gpu, lse_ref_gpu = c.fwd_gpu()
     try:
         api.fa_set_softmax_options(tau, poly)
         o, lse = c.fwd_gpu()
     finally:
-        api.fa_set_softmax_options(8.0, 0)
+        api.fa_set_softmax_options(8.0, -1)
     check_fwd(c, o, lse, all_heads(c), 128, f"variant tau={tau} poly={poly}")
     assert float((o.float() - o_ref_gpu.float()).abs().max()) <= TOL_O
     assert float((lse - lse_ref_gpu).abs().max()) <= TOL_LSE

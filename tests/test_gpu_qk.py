@@ -20,7 +20,7 @@ def _device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     build.build()
-    api.fa_set_softmax_options(8.0, 0)
+    api.fa_set_softmax_options(8.0, -1)
     yield
     torch.cuda.synchronize()
     assert api.fa_last_device_status() == (0, 0)

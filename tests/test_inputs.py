@@ -41,3 +41,13 @@ def test_attention_inputs_shapes_and_stress():
     u = I.normal(I.seed_for(3, "u"), 64); u /= np.linalg.norm(u)
     proj = q @ u
     assert 2.5 < proj.mean() < 5.5 and proj.max() > 6.0
+
+
+def test_head_inputs_equal_slices_of_the_full_tensors():
+    B, H, N, d = 2, 3, 96, 64
+    for stress in (False, True):
+        full = I.attention_inputs(7, B, H, N, d, stress=stress, with_do=True)
+        for (b, h) in ((0, 0), (1, 2), (0, 2)):
+            one = I.head_inputs(7, B, H, N, d, b, h, stress=stress, with_do=True)
+            for k in ("q", "k", "v", "do"):
+                assert np.array_equal(one[k], full[k][b, h]), (stress, b, h, k)

@@ -40,7 +40,9 @@ def _rel(a, b):
     return float((a - b).norm() / b.norm())
 
 
-@pytest.mark.parametrize("B,H,N,d,causal", [(1, 4, 1000, 128, True), (2, 3, 640, 64, False)])
+# the last case fills the scratch array to within 16 KB: 16 x 8064 = 129,024 rows at d = 128
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 4, 1000, 128, True), (2, 3, 640, 64, False),
+                                            (1, 16, 8064, 128, True)])
 def test_noalloc_matches_fa_bwd_twice(B, H, N, d, causal):
     c = Case(B, H, N, d, causal, seed_workload=21, bwd=True)
     o, lse = c.fwd_gpu()
@@ -64,3 +66,15 @@ def test_noalloc_refuses_problems_beyond_the_scratch():
     # B=1, H=16, N=32768, d=128 needs 272 MB of workspace: refused on the host, nothing launched
     rc = lib.fa_bwd_noalloc(fake, fake, fake, fake, fake, fake, fake, fake, fake, 1, 16, 32768, 128, 0.088, 1, None)
     assert rc == _lib.FA_ERR_UNSUPPORTED
+
+
+def test_noalloc_limit_is_exact():
+    lib = _lib.lib()
+    limit = 64 << 20  # FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h
+    # the largest problem at d = 128 fits, one more 128-row tile does not
+    assert lib.fa_bwd_workspace_size(1, 16, 8064, 128) <= limit
+    assert lib.fa_bwd_workspace_size(1, 1, 129024 + 128, 128) > limit
+    fake = ctypes.c_void_p(0x100000)
+    for shape in ((1, 1, 129024 + 128, 128), (1, 16, 8065, 128), (1, 2, 254080 // 2 + 128, 64)):
+        rc = lib.fa_bwd_noalloc(fake, fake, fake, fake, fake, fake, fake, fake, fake, *shape, 0.088, 1, None)
+        assert rc == _lib.FA_ERR_UNSUPPORTED, shape
