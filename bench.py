@@ -370,7 +370,10 @@ def run_gpu(args):
     }
     if not args.no_per_config:
         # every rank times the same extra shapes; rank 0 reports its own numbers (untimed by the main loop)
-        result["per_config"] = gpu_per_config(api, reps=args.per_config_reps)
+        try:
+            result["per_config"] = gpu_per_config(api, reps=args.per_config_reps)
+        except Exception as exc:  # the headline line above stands on its own
+            result["per_config"] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     if world > 1:
@@ -429,6 +432,8 @@ def gpu_per_config(api, reps=5):
 
         def timed(fn, prof_which=None):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            for e in ev[2:]:  # torch creates an event's handle at its first record
+                e.record(stream)
             flush.zero_()
             if prof_which is not None:
                 api.fa_profile_next(prof_which, ev[2], ev[3])

@@ -29,8 +29,14 @@ SIGNATURES = {
     "fa_bwd_qk_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fa_bwd_qk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _I, _I,
                        ctypes.c_float, _I, _P]),
+    "fa_fwd_accumulate": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _I, _P]),
+    "fa_bwd_prepare": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _P]),
+    "fa_bwd_accumulate": (_I, [_P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P, _I, _I, _I, _I, _I, _I,
+                               ctypes.c_float, _I, _I, _P]),
+    "fa_bwd_finish": (_I, [_P, ctypes.c_size_t, _P, _I, _I, _I, _I, ctypes.c_float, _P]),
     "fa_lse_merge": (_I, [_P, _P, _P, _P, ctypes.c_int64, _I, _I, _P]),
     "fa_accumulate_bf16": (_I, [_P, _P, ctypes.c_int64, _I, _P]),
+    "fa_accumulate_f32": (_I, [_P, _P, ctypes.c_int64, _P]),
     "fa_convert_f32_bf16": (_I, [_P, _P, ctypes.c_int64, _P]),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_last_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),

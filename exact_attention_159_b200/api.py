@@ -168,6 +168,69 @@ def fa_bwd_qk(q, k, v, o, do, lse, scale: float | None = None, causal: bool = Fa
     return dq, dk, dv
 
 
+def fa_fwd_accumulate(q, k, v, o_acc, lse_acc, scale: float | None = None, causal: bool = False,
+                      first: bool = False, stream=None) -> None:
+    """Fold attention of q over one key block (k, v) into fp32 accumulators o_acc [B, Hq, Nq, d],
+    lse_acc [B, Hq, Nq] by their log-sum-exp (first: initialise them)."""
+    B, Hq, Hkv, Nq, Nk, d = _shape_qk(q, k)
+    _need(q, "q", _BF16, (B, Hq, Nq, d))
+    for t, nm in ((k, "k"), (v, "v")):
+        _need(t, nm, _BF16, (B, Hkv, Nk, d))
+    _need(o_acc, "o_acc", torch.float32, (B, Hq, Nq, d))
+    _need(lse_acc, "lse_acc", torch.float32, (B, Hq, Nq))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    check(_lib.lib().fa_fwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, Hq, Hkv, Nq, Nk,
+                                       d, scale, int(bool(causal)), int(bool(first)), _stream(stream)),
+          "fa_fwd_accumulate")
+
+
+def fa_bwd_prepare(o, do, lse, workspace=None, stream=None):
+    """D and LSE*log2(e) of a query block into a (new or given) workspace, dQ accumulator zeroed;
+    o, do bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq].  Returns the workspace."""
+    B, Hq, Nq, d = _shape(o)
+    for t, nm in ((o, "o"), (do, "do")):
+        _need(t, nm, _BF16, (B, Hq, Nq, d))
+    _need(lse, "lse", torch.float32, (B, Hq, Nq))
+    ws_bytes = fa_bwd_qk_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=o.device)
+    _need_workspace(workspace, ws_bytes)
+    check(_lib.lib().fa_bwd_prepare(_ptr(o), _ptr(do), _ptr(lse), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), B, Hq, Nq, d, _stream(stream)),
+          "fa_bwd_prepare")
+    return workspace
+
+
+def fa_bwd_accumulate(q, k, v, do, workspace, dk_acc, dv_acc, scale: float | None = None, causal: bool = False,
+                      first: bool = False, stream=None) -> None:
+    """Gradients of one key block: dQ added into the workspace, dK (scaled) and dV stored (first) or
+    added into the fp32 accumulators dk_acc, dv_acc [B, Hkv, Nk, d]."""
+    B, Hq, Hkv, Nq, Nk, d = _shape_qk(q, k)
+    for t, nm in ((q, "q"), (do, "do")):
+        _need(t, nm, _BF16, (B, Hq, Nq, d))
+    for t, nm in ((k, "k"), (v, "v")):
+        _need(t, nm, _BF16, (B, Hkv, Nk, d))
+    for t, nm in ((dk_acc, "dk_acc"), (dv_acc, "dv_acc")):
+        _need(t, nm, torch.float32, (B, Hkv, Nk, d))
+    _need_workspace(workspace, fa_bwd_qk_workspace_size(B, Hq, Nq, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    check(_lib.lib().fa_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _ptr(dk_acc), _ptr(dv_acc),
+                                       B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), int(bool(first)),
+                                       _stream(stream)), "fa_bwd_accumulate")
+
+
+def fa_bwd_finish(workspace, B: int, Hq: int, Nq: int, d: int, scale: float | None = None, out=None, stream=None):
+    """dQ (bf16 [B, Hq, Nq, d]) from the workspace's accumulator."""
+    _need_workspace(workspace, fa_bwd_qk_workspace_size(B, Hq, Nq, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty((B, Hq, Nq, d), dtype=_BF16, device=workspace.device) if out is None else out
+    _need(out, "out", _BF16, (B, Hq, Nq, d))
+    check(_lib.lib().fa_bwd_finish(_ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(out), B, Hq,
+                                   Nq, d, scale, _stream(stream)), "fa_bwd_finish")
+    return out
+
+
 def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, first: bool = False, stream=None) -> None:
     """Fold a partial (O bf16 [..., d], LSE fp32 [...]) over one key set into an fp32 accumulator."""
     d = int(o_part.shape[-1])
@@ -186,6 +249,13 @@ def fa_accumulate_bf16(acc, x, first: bool = False, stream=None) -> None:
     _need(x, "x", _BF16, tuple(x.shape))
     check(_lib.lib().fa_accumulate_bf16(_ptr(acc), _ptr(x), x.numel(), int(bool(first)), _stream(stream)),
           "fa_accumulate_bf16")
+
+
+def fa_accumulate_f32(acc, x, stream=None) -> None:
+    """acc (fp32) += x (fp32), elementwise."""
+    _need(acc, "acc", torch.float32, tuple(x.shape))
+    _need(x, "x", torch.float32, tuple(x.shape))
+    check(_lib.lib().fa_accumulate_f32(_ptr(acc), _ptr(x), x.numel(), _stream(stream)), "fa_accumulate_f32")
 
 
 def fa_convert_f32_bf16(x, out=None, stream=None):

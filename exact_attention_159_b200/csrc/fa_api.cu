@@ -94,22 +94,66 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// Encoded tensor maps of recent calls, keyed by (address, extents, box, element kind): callers that
+// reuse their buffers (training loops, graph replays, the ring steps) skip cuTensorMapEncodeTiled.
+// A map holds only the address and geometry it was encoded from, so a hit is exactly the map a
+// fresh encode would produce.  Small, round-robin replacement, one lock.
+struct MapKey {
+  const void* base;
+  int BH, N, d, rows, kind;  // kind 0: bf16 operand, 1: fp32 dQ accumulator
+  bool operator==(const MapKey& o) const {
+    return base == o.base && BH == o.BH && N == o.N && d == o.d && rows == o.rows && kind == o.kind;
+  }
+};
+struct MapCache {
+  static constexpr int kSlots = 64;
+  std::mutex mu;
+  MapKey key[kSlots] = {};
+  CUtensorMap map[kSlots];
+  int used = 0, next = 0;
+};
+MapCache g_maps;
+
+bool map_lookup(const MapKey& k, CUtensorMap* out) {
+  std::lock_guard<std::mutex> lock(g_maps.mu);
+  for (int i = 0; i < g_maps.used; ++i)
+    if (g_maps.key[i] == k) {
+      *out = g_maps.map[i];
+      return true;
+    }
+  return false;
+}
+void map_store(const MapKey& k, const CUtensorMap& m) {
+  std::lock_guard<std::mutex> lock(g_maps.mu);
+  const int i = g_maps.used < MapCache::kSlots ? g_maps.used++ : g_maps.next;
+  if (i == g_maps.next) g_maps.next = (g_maps.next + 1) % MapCache::kSlots;
+  g_maps.key[i] = k;
+  g_maps.map[i] = m;
+}
+
 // 3-D map over a contiguous [BH, N, d] bf16 tensor: box 64 (d) x `rows` x 1, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, int BH, int N, int d, int rows = 128) {
+  const MapKey key{base, BH, N, d, rows, 0};
+  if (map_lookup(key, map)) return true;
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_store(key, *map);
+  return true;
 }
 
 // 3-D map over the fp32 dQ accumulator [BH, Npad, d]: box 32 (d) x `rows` x 1, 128-byte swizzle
 // (the layout of the backward kernels' staging buffers for their TMA reduce-add).
 bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d, int rows = 128) {
+  const MapKey key{base, BH, npad, d, rows, 1};
+  if (map_lookup(key, map)) return true;
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(npad),
@@ -117,9 +161,12 @@ bool make_acc_map(CUtensorMap* map, void* base, int BH, int npad, int d, int row
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(npad) * d * 4};
   const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  map_store(key, *map);
+  return true;
 }
 
 // Shape checks shared by forward and backward (Hq query heads over Hkv key/value heads, Nq query
@@ -147,9 +194,28 @@ int check_shape(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int 
   return FA_OK;
 }
 
+// The dynamic shared memory limit of a kernel is a per-device attribute: set it once per (kernel,
+// device) and remember that it is set.
+std::mutex g_attr_mu;
+struct AttrDone {
+  const void* kernel;
+  int device;
+};
+AttrDone g_attr_done[256];
+int g_attr_count = 0;
+
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (int i = 0; i < g_attr_count; ++i)
+    if (g_attr_done[i].kernel == key && g_attr_done[i].device == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && g_attr_count < 256) g_attr_done[g_attr_count++] = AttrDone{key, dev};
+  return e;
 }
 
 template <int D, bool C, int P>
@@ -273,6 +339,163 @@ __global__ void exp2_eval_kernel(const float* __restrict__ x, float* __restrict_
   }
 }
 
+// True when any of the `no` output ranges overlaps an input range or another output range.
+bool any_overlap(const void* const* outs, const size_t* osz, int no, const void* const* ins, const size_t* isz, int ni) {
+  for (int a = 0; a < no; ++a) {
+    for (int b = 0; b < ni; ++b)
+      if (overlaps(outs[a], osz[a], ins[b], isz[b])) return true;
+    for (int b = a + 1; b < no; ++b)
+      if (overlaps(outs[a], osz[a], outs[b], osz[b])) return true;
+  }
+  return false;
+}
+
+// The forward after its argument checks: bf16 O and LSE, or (O_acc non-null) the fold into fp32
+// accumulators.  The cluster-pair variant serves only plain bf16 calls.
+int fwd_launch(const void* Q, const void* K, const void* V, void* O, float* LSE, float* O_acc, float* LSE_acc,
+               int acc_first, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+  int rc = FA_OK;
+  int* status = device_status(&rc);
+  if (!status) return rc;
+  const int BH = B * Hq, BHkv = B * Hkv;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d))
+    return FA_ERR_CUDA;
+  fa::FwdParams prm;
+  prm.O = static_cast<__nv_bfloat16*>(O);
+  prm.LSE = LSE;
+  prm.O_acc = O_acc;
+  prm.LSE_acc = LSE_acc;
+  prm.acc_first = acc_first;
+  prm.N = Nq;
+  prm.Nk = Nk;
+  prm.BH = BH;
+  prm.Hq = Hq;
+  prm.G = Hq / Hkv;
+  prm.off = Nk - Nq;
+  const int tiles = (Nq + 127) / 128;
+  prm.n_pairs = (tiles + 1) / 2;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.tau = g_tau.load(std::memory_order_relaxed);
+  prm.status = status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int poly_set = g_poly.load(std::memory_order_relaxed);
+  const int poly = poly_set >= 0 ? poly_set : kPolyDefault[d == 128 ? 1 : 0];
+  if (!O_acc && d == 128 && g_fwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
+    CUtensorMap mk64;
+    if (!make_map(&mk64, K, BH, Nk, d, 64)) return FA_ERR_CUDA;
+    fa::Fwd2Params p2;
+    p2.O = prm.O;
+    p2.LSE = prm.LSE;
+    p2.N = Nq;
+    p2.BH = BH;
+    p2.n_quads = (tiles + 3) / 4;
+    p2.scale_log2 = prm.scale_log2;
+    p2.tau = prm.tau;
+    p2.status = prm.status;
+    const bool prof2 = prof_begin(0, st);
+    rc = causal ? launch_fwd2_poly<true>(poly, mq, mk64, mv, p2, st) : launch_fwd2_poly<false>(poly, mq, mk64, mv, p2, st);
+    if (prof2) prof_end(0, st);
+    return rc;
+  }
+  const bool prof = prof_begin(0, st);
+  if (d == 128)
+    rc = causal ? launch_fwd_poly<128, true>(poly, mq, mk, mv, prm, st)
+                : launch_fwd_poly<128, false>(poly, mq, mk, mv, prm, st);
+  else
+    rc = causal ? launch_fwd_poly<64, true>(poly, mq, mk, mv, prm, st)
+                : launch_fwd_poly<64, false>(poly, mq, mk, mv, prm, st);
+  if (prof) prof_end(0, st);
+  return rc;
+}
+
+// Backward step 1: -D_i, -LSE_i * log2(e) for every (padded) query row and the fp32 dQ accumulator
+// zeroed, all in the workspace.
+int bwd_prep_launch(const void* O, const void* dO, const float* LSE, uint8_t* wsb, const WsLayout& ws, int BH, int Nq,
+                    int d, cudaStream_t st) {
+  const int npad = (Nq + 127) / 128 * 128;
+  const long long prep_rows = static_cast<long long>(BH) * npad;
+  const unsigned prep_grid = static_cast<unsigned>((prep_rows * (d / 8) + 255) / 256);
+  float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
+  float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
+  float* dsum = reinterpret_cast<float*>(wsb + ws.dsum);
+  const auto* o = static_cast<const __nv_bfloat16*>(O);
+  const auto* g = static_cast<const __nv_bfloat16*>(dO);
+  if (d == 128)
+    fa::bwd_prep_kernel<128><<<prep_grid, 256, 0, st>>>(o, g, LSE, lse2, dsum, dq_acc, Nq, npad, prep_rows);
+  else
+    fa::bwd_prep_kernel<64><<<prep_grid, 256, 0, st>>>(o, g, LSE, lse2, dsum, dq_acc, Nq, npad, prep_rows);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Backward step 2: the main kernel over one key block.  dQ adds into the workspace accumulator;
+// dK and dV are written as bf16 (dK, dV) or added to fp32 accumulators (dK_acc, dV_acc).
+int bwd_main_launch(const void* Q, const void* K, const void* V, const void* dO, uint8_t* wsb, const WsLayout& ws,
+                    void* dK, void* dV, float* dK_acc, float* dV_acc, int acc_first, int B, int Hq, int Hkv, int Nq,
+                    int Nk, int d, float scale, int causal, int* status, cudaStream_t st, bool allow_pair) {
+  const int BH = B * Hq, BHkv = B * Hkv;
+  const int q_tiles = (Nq + 127) / 128;
+  const int npad = q_tiles * 128;
+  float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
+  CUtensorMap mq, mk, mv, mdo, macc;
+  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d) ||
+      !make_map(&mdo, dO, BH, Nq, d) || !make_acc_map(&macc, dq_acc, BH, npad, d))
+    return FA_ERR_CUDA;
+  fa::BwdParams prm;
+  prm.nlse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
+  prm.ndsum = reinterpret_cast<const float*>(wsb + ws.dsum);
+  prm.dK = static_cast<__nv_bfloat16*>(dK);
+  prm.dV = static_cast<__nv_bfloat16*>(dV);
+  prm.dK_acc = dK_acc;
+  prm.dV_acc = dV_acc;
+  prm.acc_first = acc_first;
+  prm.N = Nq;
+  prm.Npad = npad;
+  prm.Nk = Nk;
+  prm.BHkv = BHkv;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.off = Nk - Nq;
+  prm.n_q_tiles = q_tiles;
+  prm.n_kv_tiles = (Nk + 127) / 128;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.scale = scale;
+  prm.status = status;
+  int rc = FA_OK;
+  const bool prof = prof_begin(1, st);
+  if (allow_pair && d == 128 && g_bwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
+    CUtensorMap mq64, mdo64, macc64;
+    if (!make_map(&mq64, Q, BH, Nq, d, 64) || !make_map(&mdo64, dO, BH, Nq, d, 64) ||
+        !make_acc_map(&macc64, dq_acc, BH, npad, d, 64))
+      rc = FA_ERR_CUDA;
+    else
+      rc = causal ? launch_bwd2<true>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st)
+                  : launch_bwd2<false>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st);
+  } else if (d == 128) {
+    rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, macc, prm, st)
+                : launch_bwd<128, false>(mq, mk, mv, mdo, macc, prm, st);
+  } else {
+    rc = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, macc, prm, st)
+                : launch_bwd<64, false>(mq, mk, mv, mdo, macc, prm, st);
+  }
+  if (prof) prof_end(1, st);
+  return rc;
+}
+
+// Backward step 3: dQ = bf16(scale * dQ_acc) for the real rows.
+int bwd_finish_launch(uint8_t* wsb, const WsLayout& ws, void* dQ, int BH, int Nq, int d, float scale, cudaStream_t st) {
+  const int npad = (Nq + 127) / 128 * 128;
+  const float* dq_acc = reinterpret_cast<const float*>(wsb + ws.dq);
+  const long long rows = static_cast<long long>(BH) * Nq;
+  const unsigned cgrid = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
+  if (d == 128)
+    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
+  else
+    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -310,60 +533,33 @@ int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, float* LSE, 
   const int BH = B * Hq, BHkv = B * Hkv;
   const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, kb = static_cast<size_t>(BHkv) * Nk * d * 2;
   const size_t lb = static_cast<size_t>(BH) * Nq * 4;
+  const void* outs[2] = {O, LSE};
+  const size_t osz[2] = {qb, lb};
   const void* ins[3] = {Q, K, V};
   const size_t isz[3] = {qb, kb, kb};
-  for (int i = 0; i < 3; ++i)
-    if (overlaps(O, qb, ins[i], isz[i]) || overlaps(LSE, lb, ins[i], isz[i])) return FA_ERR_INVALID_ARG;
-  if (overlaps(O, qb, LSE, lb)) return FA_ERR_INVALID_ARG;
-  int* status = device_status(&rc);
-  if (!status) return rc;
+  if (any_overlap(outs, osz, 2, ins, isz, 3)) return FA_ERR_INVALID_ARG;
+  return fwd_launch(Q, K, V, O, LSE, nullptr, nullptr, 0, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
+}
 
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d))
-    return FA_ERR_CUDA;
-  fa::FwdParams prm;
-  prm.O = static_cast<__nv_bfloat16*>(O);
-  prm.LSE = LSE;
-  prm.N = Nq;
-  prm.Nk = Nk;
-  prm.BH = BH;
-  prm.Hq = Hq;
-  prm.G = Hq / Hkv;
-  prm.off = Nk - Nq;
-  const int tiles = (Nq + 127) / 128;
-  prm.n_pairs = (tiles + 1) / 2;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.tau = g_tau.load(std::memory_order_relaxed);
-  prm.status = status;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int poly_set = g_poly.load(std::memory_order_relaxed);
-  const int poly = poly_set >= 0 ? poly_set : kPolyDefault[d == 128 ? 1 : 0];
-  if (d == 128 && g_fwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
-    CUtensorMap mk64;
-    if (!make_map(&mk64, K, BH, Nk, d, 64)) return FA_ERR_CUDA;
-    fa::Fwd2Params p2;
-    p2.O = prm.O;
-    p2.LSE = prm.LSE;
-    p2.N = Nq;
-    p2.BH = BH;
-    p2.n_quads = (tiles + 3) / 4;
-    p2.scale_log2 = prm.scale_log2;
-    p2.tau = prm.tau;
-    p2.status = prm.status;
-    const bool prof2 = prof_begin(0, st);
-    rc = causal ? launch_fwd2_poly<true>(poly, mq, mk64, mv, p2, st) : launch_fwd2_poly<false>(poly, mq, mk64, mv, p2, st);
-    if (prof2) prof_end(0, st);
-    return rc;
-  }
-  const bool prof = prof_begin(0, st);
-  if (d == 128)
-    rc = causal ? launch_fwd_poly<128, true>(poly, mq, mk, mv, prm, st)
-                : launch_fwd_poly<128, false>(poly, mq, mk, mv, prm, st);
-  else
-    rc = causal ? launch_fwd_poly<64, true>(poly, mq, mk, mv, prm, st)
-                : launch_fwd_poly<64, false>(poly, mq, mk, mv, prm, st);
-  if (prof) prof_end(0, st);
-  return rc;
+int fa_fwd_accumulate(const void* Q, const void* K, const void* V, float* O_acc, float* LSE_acc, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int causal, int first, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty);
+  if (rc != FA_OK) return rc;
+  if (first != 0 && first != 1) return FA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O_acc || !LSE_acc) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O_acc) || !aligned16(LSE_acc))
+    return FA_ERR_ALIGNMENT;
+  const int BH = B * Hq, BHkv = B * Hkv;
+  const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, kb = static_cast<size_t>(BHkv) * Nk * d * 2;
+  const size_t lb = static_cast<size_t>(BH) * Nq * 4;
+  const void* outs[2] = {O_acc, LSE_acc};
+  const size_t osz[2] = {2 * qb, lb};
+  const void* ins[3] = {Q, K, V};
+  const size_t isz[3] = {qb, kb, kb};
+  if (any_overlap(outs, osz, 2, ins, isz, 3)) return FA_ERR_INVALID_ARG;
+  return fwd_launch(Q, K, V, nullptr, nullptr, O_acc, LSE_acc, first, B, Hq, Hkv, Nq, Nk, d, scale, causal, stream);
 }
 
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B, int H, int N, int d,
@@ -399,83 +595,81 @@ int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const 
   const size_t osz[4] = {qb, kb, kb, ws.total};
   const void* ins[6] = {Q, K, V, O, dO, LSE};
   const size_t isz[6] = {qb, kb, kb, qb, qb, lb};
-  for (int a = 0; a < 4; ++a) {
-    for (int b = 0; b < 6; ++b)
-      if (overlaps(outs[a], osz[a], ins[b], isz[b])) return FA_ERR_INVALID_ARG;
-    for (int b = a + 1; b < 4; ++b)
-      if (overlaps(outs[a], osz[a], outs[b], osz[b])) return FA_ERR_INVALID_ARG;
-  }
+  if (any_overlap(outs, osz, 4, ins, isz, 6)) return FA_ERR_INVALID_ARG;
   int* status = device_status(&rc);
   if (!status) return rc;
-
-  uint8_t* wsb = static_cast<uint8_t*>(workspace);
-  const int q_tiles = (Nq + 127) / 128;
-  const int npad = q_tiles * 128;
-  float* dq_acc = reinterpret_cast<float*>(wsb + ws.dq);
-  CUtensorMap mq, mk, mv, mdo, macc;
-  if (!make_map(&mq, Q, BH, Nq, d) || !make_map(&mk, K, BHkv, Nk, d) || !make_map(&mv, V, BHkv, Nk, d) ||
-      !make_map(&mdo, dO, BH, Nq, d) || !make_acc_map(&macc, dq_acc, BH, npad, d))
-    return FA_ERR_CUDA;
-  fa::BwdParams prm;
-  prm.nlse2 = reinterpret_cast<const float*>(wsb + ws.lse2);
-  prm.ndsum = reinterpret_cast<const float*>(wsb + ws.dsum);
-  prm.dK = static_cast<__nv_bfloat16*>(dK);
-  prm.dV = static_cast<__nv_bfloat16*>(dV);
-  prm.N = Nq;
-  prm.Npad = npad;
-  prm.Nk = Nk;
-  prm.BHkv = BHkv;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.G = Hq / Hkv;
-  prm.off = Nk - Nq;
-  prm.n_q_tiles = q_tiles;
-  prm.n_kv_tiles = (Nk + 127) / 128;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.scale = scale;
-  prm.status = status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+  if ((rc = bwd_prep_launch(O, dO, LSE, wsb, ws, BH, Nq, d, st)) != FA_OK) return rc;
+  if ((rc = bwd_main_launch(Q, K, V, dO, wsb, ws, dK, dV, nullptr, nullptr, 0, B, Hq, Hkv, Nq, Nk, d, scale, causal,
+                            status, st, true)) != FA_OK)
+    return rc;
+  return bwd_finish_launch(wsb, ws, dQ, BH, Nq, d, scale, st);
+}
 
-  const long long prep_rows = static_cast<long long>(BH) * npad;
-  const long long prep_threads = prep_rows * (d / 8);
-  const unsigned prep_grid = static_cast<unsigned>((prep_threads + 255) / 256);
-  float* lse2 = reinterpret_cast<float*>(wsb + ws.lse2);
-  float* dsum = reinterpret_cast<float*>(wsb + ws.dsum);
-  if (d == 128)
-    fa::bwd_prep_kernel<128><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
-                                                        static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                        dq_acc, Nq, npad, prep_rows);
-  else
-    fa::bwd_prep_kernel<64><<<prep_grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O),
-                                                       static_cast<const __nv_bfloat16*>(dO), LSE, lse2, dsum,
-                                                       dq_acc, Nq, npad, prep_rows);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-
-  const bool prof = prof_begin(1, st);
-  if (d == 128 && g_bwd_pair.load(std::memory_order_relaxed) && Hq == Hkv && Nq == Nk) {
-    CUtensorMap mq64, mdo64, macc64;
-    if (!make_map(&mq64, Q, BH, Nq, d, 64) || !make_map(&mdo64, dO, BH, Nq, d, 64) ||
-        !make_acc_map(&macc64, dq_acc, BH, npad, d, 64))
-      rc = FA_ERR_CUDA;
-    else
-      rc = causal ? launch_bwd2<true>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st)
-                  : launch_bwd2<false>(mq, mq64, mk, mv, mdo, mdo64, macc64, prm, st);
-  } else if (d == 128)
-    rc = causal ? launch_bwd<128, true>(mq, mk, mv, mdo, macc, prm, st)
-                : launch_bwd<128, false>(mq, mk, mv, mdo, macc, prm, st);
-  else
-    rc = causal ? launch_bwd<64, true>(mq, mk, mv, mdo, macc, prm, st)
-                : launch_bwd<64, false>(mq, mk, mv, mdo, macc, prm, st);
-  if (prof) prof_end(1, st);
+int fa_bwd_prepare(const void* O, const void* dO, const float* LSE, void* workspace, size_t workspace_bytes, int B,
+                   int Hq, int Nq, int d, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, Hq, Hq, Nq, Nq, d, 1.0f, 0, &empty);
   if (rc != FA_OK) return rc;
+  if (!O || !dO || !LSE || !workspace) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  for (const void* p : {O, dO, static_cast<const void*>(LSE), static_cast<const void*>(workspace)})
+    if (!aligned16(p)) return FA_ERR_ALIGNMENT;
+  const int BH = B * Hq;
+  const WsLayout ws = ws_layout(BH, Nq, d);
+  if (workspace_bytes < ws.total) return FA_ERR_INVALID_ARG;
+  const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, lb = static_cast<size_t>(BH) * Nq * 4;
+  const void* outs[1] = {workspace};
+  const size_t osz[1] = {ws.total};
+  const void* ins[3] = {O, dO, LSE};
+  const size_t isz[3] = {qb, qb, lb};
+  if (any_overlap(outs, osz, 1, ins, isz, 3)) return FA_ERR_INVALID_ARG;
+  return bwd_prep_launch(O, dO, LSE, static_cast<uint8_t*>(workspace), ws, BH, Nq, d,
+                         static_cast<cudaStream_t>(stream));
+}
 
-  const long long rows = static_cast<long long>(BH) * Nq;
-  const unsigned cgrid = static_cast<unsigned>((rows * (d / 8) + 255) / 256);
-  if (d == 128)
-    fa::bwd_dq_kernel<128><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
-  else
-    fa::bwd_dq_kernel<64><<<cgrid, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), scale, Nq, npad, rows);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+int fa_bwd_accumulate(const void* Q, const void* K, const void* V, const void* dO, void* workspace,
+                      size_t workspace_bytes, float* dK_acc, float* dV_acc, int B, int Hq, int Hkv, int Nq, int Nk,
+                      int d, float scale, int causal, int first, void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty);
+  if (rc != FA_OK) return rc;
+  if (first != 0 && first != 1) return FA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !dO || !workspace || !dK_acc || !dV_acc) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  for (const void* p : {Q, K, V, dO, static_cast<const void*>(workspace), static_cast<const void*>(dK_acc),
+                        static_cast<const void*>(dV_acc)})
+    if (!aligned16(p)) return FA_ERR_ALIGNMENT;
+  const int BH = B * Hq, BHkv = B * Hkv;
+  const WsLayout ws = ws_layout(BH, Nq, d);
+  if (workspace_bytes < ws.total) return FA_ERR_INVALID_ARG;
+  const size_t qb = static_cast<size_t>(BH) * Nq * d * 2, kb = static_cast<size_t>(BHkv) * Nk * d * 2;
+  const void* outs[3] = {workspace, dK_acc, dV_acc};
+  const size_t osz[3] = {ws.total, 2 * kb, 2 * kb};
+  const void* ins[4] = {Q, K, V, dO};
+  const size_t isz[4] = {qb, kb, kb, qb};
+  if (any_overlap(outs, osz, 3, ins, isz, 4)) return FA_ERR_INVALID_ARG;
+  int* status = device_status(&rc);
+  if (!status) return rc;
+  return bwd_main_launch(Q, K, V, dO, static_cast<uint8_t*>(workspace), ws, nullptr, nullptr, dK_acc, dV_acc, first, B,
+                         Hq, Hkv, Nq, Nk, d, scale, causal, status, static_cast<cudaStream_t>(stream), false);
+}
+
+int fa_bwd_finish(void* workspace, size_t workspace_bytes, void* dQ, int B, int Hq, int Nq, int d, float scale,
+                  void* stream) {
+  bool empty = false;
+  int rc = check_shape(B, Hq, Hq, Nq, Nq, d, scale, 0, &empty);
+  if (rc != FA_OK) return rc;
+  if (!workspace || !dQ) return FA_ERR_INVALID_ARG;
+  if (empty) return FA_OK;
+  if (!aligned16(workspace) || !aligned16(dQ)) return FA_ERR_ALIGNMENT;
+  const int BH = B * Hq;
+  const WsLayout ws = ws_layout(BH, Nq, d);
+  if (workspace_bytes < ws.total) return FA_ERR_INVALID_ARG;
+  if (overlaps(dQ, static_cast<size_t>(BH) * Nq * d * 2, workspace, ws.total)) return FA_ERR_INVALID_ARG;
+  return bwd_finish_launch(static_cast<uint8_t*>(workspace), ws, dQ, BH, Nq, d, scale,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
@@ -588,6 +782,16 @@ int fa_accumulate_bf16(float* acc, const void* x, int64_t n, int first, void* st
   if (overlaps(acc, static_cast<size_t>(n) * 4, x, static_cast<size_t>(n) * 2)) return FA_ERR_INVALID_ARG;
   fa::accumulate_bf16_kernel<<<elementwise_grid(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       acc, static_cast<const __nv_bfloat16*>(x), n / 8, first);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_accumulate_f32(float* acc, const float* x, int64_t n, void* stream) {
+  if (n < 0 || (n & 7)) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!acc || !x) return FA_ERR_INVALID_ARG;
+  if (!aligned16(acc) || !aligned16(x)) return FA_ERR_ALIGNMENT;
+  if (overlaps(acc, static_cast<size_t>(n) * 4, x, static_cast<size_t>(n) * 4)) return FA_ERR_INVALID_ARG;
+  fa::accumulate_f32_kernel<<<elementwise_grid(n / 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(acc, x, n / 8);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -37,8 +37,11 @@ namespace fa {
 struct BwdParams {
   const float* nlse2;  // [B * Hq, Npad]  -LSE * log2(e); -inf on padding rows and rows that see no key
   const float* ndsum;  // [B * Hq, Npad]  -D_i, 0 on padding rows
-  __nv_bfloat16* dK;   // [B * Hkv, Nk, D]
+  __nv_bfloat16* dK;   // [B * Hkv, Nk, D]  (bf16 outputs, when dK_acc is null)
   __nv_bfloat16* dV;   // [B * Hkv, Nk, D]
+  float* dK_acc;       // [B * Hkv, Nk, D] fp32 accumulators: when set, dK (x scale) and dV are added
+  float* dV_acc;       // to them (or stored, when acc_first) instead of written as bf16
+  int acc_first;
   int N, Npad;         // query rows per head, padded to whole tiles
   int Nk;              // key rows per head
   int BHkv, Hq, Hkv, G;  // batch * key/value heads; heads per batch entry; query heads per key/value head
@@ -392,6 +395,35 @@ __global__ void __launch_bounds__(384, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = tmem + (which == 0 ? L::kColDK : L::kColDV) + lane_off;
         const float mul = which == 0 ? prm.scale : 1.0f;
+        if (prm.dK_acc != nullptr) {
+          // fp32 accumulators (gradients of one query block summed over several calls); each key
+          // row belongs to exactly one CTA, so the read-modify-write needs no atomics
+          float* acc_row = (which == 0 ? prm.dK_acc : prm.dV_acc) + rowoff;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t a[32];
+            tmem_ld32(tcol + 32 * c, a);
+            tmem_wait_ld();
+            reg_fence(a);
+            if (store) {
+              float4* dst = reinterpret_cast<float4*>(acc_row + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                float4 v = make_float4(__uint_as_float(a[4 * i]) * mul, __uint_as_float(a[4 * i + 1]) * mul,
+                                       __uint_as_float(a[4 * i + 2]) * mul, __uint_as_float(a[4 * i + 3]) * mul);
+                if (!prm.acc_first) {
+                  const float4 o = dst[i];
+                  v.x += o.x;
+                  v.y += o.y;
+                  v.z += o.z;
+                  v.w += o.w;
+                }
+                dst[i] = v;
+              }
+            }
+          }
+          continue;
+        }
         __nv_bfloat16* dst_row = (which == 0 ? prm.dK : prm.dV) + rowoff;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

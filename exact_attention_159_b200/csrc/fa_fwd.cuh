@@ -50,6 +50,9 @@ enum : int { kSiteFwd = 0x100, kSiteBwd = 0x200 };
 struct FwdParams {
   __nv_bfloat16* O;   // [BH, N, D]
   float* LSE;         // [BH, N], natural log
+  float* O_acc;       // [BH, N, D] fp32: when set, this call's (O, LSE) is folded into (O_acc, LSE_acc)
+  float* LSE_acc;     // [BH, N]       by their log-sum-exp instead of being written to O, LSE
+  int acc_first;      // 1: the accumulators are initialised from this call
   int N;              // query rows per head
   int Nk;             // key rows per head
   int BH;             // batch * query heads
@@ -375,6 +378,7 @@ __global__ void __launch_bounds__(640, 1)
       tc_fence_before();
       if (ok) mbar_arrive(&p_full[t]);
     }
+    float lse_old = -INFINITY;  // accumulating calls: the row's LSE over the key blocks folded so far
     if (nkv[t] > 0) {
       // full row sum from the two halves (joint decision, as in the loop)
       const bool okl = ok && wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
@@ -382,9 +386,52 @@ __global__ void __launch_bounds__(640, 1)
         tc_fence_after();
         xchg[128 * h + r] = l;
       }
+      // both threads of the row read the old LSE before the barrier; it is replaced after it
+      if (prm.O_acc != nullptr && !prm.acc_first && row < prm.N)
+        lse_old = prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row];
       ok = group_and(bar_id, 64, okl);
     }
-    if (ok && nkv[t] > 0) {
+    if (ok && nkv[t] > 0 && prm.O_acc != nullptr) {
+      // fold into the fp32 accumulators: L = ln(e^LSE_old + e^LSE), O_acc = e^(LSE_old - L) O_acc +
+      // e^(LSE - L) O (a side at -inf weighs 0; both at -inf leave O_acc = 0, LSE_acc = -inf)
+      const float l_row = l + xchg[128 * (h ^ 1) + r];
+      const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+      const bool store = row < prm.N;
+      const float lse = l_row > 0.0f ? (m_ref + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+      float lse_new = lse, wa = 0.0f, wb = 1.0f;
+      if (!prm.acc_first) {
+        const float mx = fmaxf(lse_old, lse);
+        lse_new = mx == -INFINITY ? -INFINITY : mx + log1pf(expf(-fabsf(lse_old - lse)));
+        wa = lse_new == -INFINITY ? 0.0f : expf(lse_old - lse_new);
+        wb = lse_new == -INFINITY ? 0.0f : expf(lse - lse_new);
+      }
+      const float scale_b = inv_l * wb;
+      float* arow = prm.O_acc + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D + (D / 2) * h;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        if (store) {
+          float4* dst = reinterpret_cast<float4*>(arow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 v = make_float4(__uint_as_float(o[4 * i]) * scale_b, __uint_as_float(o[4 * i + 1]) * scale_b,
+                                   __uint_as_float(o[4 * i + 2]) * scale_b, __uint_as_float(o[4 * i + 3]) * scale_b);
+            if (!prm.acc_first) {
+              const float4 a = dst[i];
+              v.x = fmaf(wa, a.x, v.x);
+              v.y = fmaf(wa, a.y, v.y);
+              v.z = fmaf(wa, a.z, v.z);
+              v.w = fmaf(wa, a.w, v.w);
+            }
+            dst[i] = v;
+          }
+        }
+      }
+      if (store && h == 0) prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row] = lse_new;
+    } else if (ok && nkv[t] > 0) {
       const float l_row = l + xchg[128 * (h ^ 1) + r];
       const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;  // a row that sees no key: O = 0, LSE = -inf
       const bool store = row < prm.N;
@@ -409,11 +456,19 @@ __global__ void __launch_bounds__(640, 1)
         prm.LSE[static_cast<size_t>(bh) * prm.N + row] =
             l_row > 0.0f ? (m_ref + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     } else if (nkv[t] == 0 && qt < n_tiles && row < prm.N) {
-      // a query tile no key is visible to (causal, N > Nk): O = 0, LSE = -inf
-      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
+      // a query tile no key is visible to (causal, N > Nk): O = 0, LSE = -inf (an accumulating call
+      // that is not the first adds nothing)
+      if (prm.O_acc == nullptr) {
+        __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
 #pragma unroll
-      for (int i = 0; i < D / 16; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0u, 0u, 0u, 0u);
-      if (h == 0) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
+        for (int i = 0; i < D / 16; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (h == 0) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
+      } else if (prm.acc_first) {
+        float* arow = prm.O_acc + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<float4*>(arow)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (h == 0) prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
+      }
     }
   }
 

@@ -88,6 +88,20 @@ __global__ void __launch_bounds__(256) accumulate_bf16_kernel(float* __restrict_
   }
 }
 
+// acc (fp32, n) += x (fp32, n); n a multiple of 8.
+__global__ void __launch_bounds__(256) accumulate_f32_kernel(float* __restrict__ acc, const float* __restrict__ x,
+                                                             long long n8) {
+  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < n8;
+       t += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(x + t * 8);
+    float4* a = reinterpret_cast<float4*>(acc + t * 8);
+    const float4 x0 = src[0], x1 = src[1];
+    float4 a0 = a[0], a1 = a[1];
+    a[0] = make_float4(a0.x + x0.x, a0.y + x0.y, a0.z + x0.z, a0.w + x0.w);
+    a[1] = make_float4(a1.x + x1.x, a1.y + x1.y, a1.z + x1.z, a1.w + x1.w);
+  }
+}
+
 // y (bf16, n) = round-to-nearest-even(x (fp32, n)); n a multiple of 8.
 __global__ void __launch_bounds__(256) convert_f32_bf16_kernel(const float* __restrict__ x,
                                                                __nv_bfloat16* __restrict__ y, long long n8) {

@@ -122,6 +122,58 @@ int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const 
               int d, float scale, int causal, void* stream);
 
 /*
+ * Forward over one block of keys, folded into running fp32 results, for
+ * callers that attend one block of query rows to several key blocks in turn
+ * (ring / context parallelism).  Q bf16 [B, Hq, Nq, d]; K, V bf16
+ * [B, Hkv, Nk, d] (masked as fa_fwd_qk masks them).  O_acc fp32
+ * [B, Hq, Nq, d] and LSE_acc fp32 [B, Hq, Nq] hold the result over the key
+ * blocks folded so far; with this block's O_b, LSE_b the kernel writes
+ * L = ln(exp(LSE_acc) + exp(LSE_b)), O_acc = exp(LSE_acc - L) O_acc +
+ * exp(LSE_b - L) O_b, which is exact attention over the union of the blocks
+ * (the per-row log-sum-exp that the online softmax uses across key tiles,
+ * one level up).  first = 1 initialises the accumulators from this block
+ * (their old contents are not read).  A side whose LSE is -inf weighs
+ * nothing; rows that see no key in any block end with O_acc = 0, LSE_acc =
+ * -inf.  No bf16 rounding happens between blocks.  One launch; checks and
+ * status codes as fa_fwd_qk (first must be 0 or 1, every pointer 16-byte
+ * aligned, the accumulators may not overlap the inputs).
+ */
+int fa_fwd_accumulate(const void* Q, const void* K, const void* V, float* O_acc, float* LSE_acc, int B, int Hq,
+                      int Hkv, int Nq, int Nk, int d, float scale, int causal, int first, void* stream);
+
+/*
+ * The backward in three steps, for callers that sum the gradients of one
+ * block of query rows over several blocks of keys (ring / context
+ * parallelism, where the key blocks arrive one at a time): the result over
+ * the union of key blocks equals fa_bwd_qk over the whole key set, with no
+ * rounding to bf16 between blocks.  The rows' O and LSE must be the final ones
+ * over the whole key set (P is recomputed from LSE, and D from O and dO).
+ *
+ * fa_bwd_prepare: O, dO bf16 [B, Hq, Nq, d], LSE fp32 [B, Hq, Nq] (read).
+ *   Writes D = rowsum(dO * O) and LSE * log2(e) into the workspace (at least
+ *   fa_bwd_qk_workspace_size(B, Hq, Nq, d) bytes) and zeroes its fp32 dQ
+ *   accumulator.  One launch.
+ * fa_bwd_accumulate: Q, dO bf16 [B, Hq, Nq, d]; K, V bf16 [B, Hkv, Nk, d]
+ *   (one key block, masked as fa_bwd_qk masks it: causal aligns the last
+ *   query with the last key of THIS block).  Adds this block's dQ into the
+ *   workspace accumulator; dK_acc, dV_acc fp32 [B, Hkv, Nk, d] receive the
+ *   block's dK (scaled) and dV: stored when first = 1, added when first = 0.
+ *   One launch; the workspace must come from fa_bwd_prepare of the same query
+ *   block and must not be shared by calls that may overlap on the GPU.
+ * fa_bwd_finish: dQ bf16 [B, Hq, Nq, d] = scale * the accumulated dQ.  One
+ *   launch.
+ * Same checks and status codes as fa_bwd_qk (first must be 0 or 1); every
+ * pointer 16-byte aligned; outputs may not overlap inputs.
+ */
+int fa_bwd_prepare(const void* O, const void* dO, const float* LSE, void* workspace, size_t workspace_bytes, int B,
+                   int Hq, int Nq, int d, void* stream);
+int fa_bwd_accumulate(const void* Q, const void* K, const void* V, const void* dO, void* workspace,
+                      size_t workspace_bytes, float* dK_acc, float* dV_acc, int B, int Hq, int Hkv, int Nq, int Nk,
+                      int d, float scale, int causal, int first, void* stream);
+int fa_bwd_finish(void* workspace, size_t workspace_bytes, void* dQ, int B, int Hq, int Nq, int d, float scale,
+                  void* stream);
+
+/*
  * Pieces of ring (context-parallel) attention, where each GPU holds one
  * chunk of the sequence and the key/value chunks travel around the ring of
  * GPUs (the pages name multi-card use for long contexts -- "NVIDIA Blackwell:
@@ -144,6 +196,13 @@ int fa_lse_merge(const void* O_part, const float* LSE_part, float* O_acc, float*
 
 /* acc (fp32, n) = (first ? 0 : acc) + x (bf16, n); n a multiple of 8, both 16-byte aligned. */
 int fa_accumulate_bf16(float* acc, const void* x, int64_t n, int first, void* stream);
+
+/*
+ * acc (fp32, n) += x (fp32, n), elementwise: adds one step's gradient block to
+ * an accumulator (ring backward).  n a multiple of 8, both 16-byte aligned,
+ * not overlapping.  One launch on `stream`.
+ */
+int fa_accumulate_f32(float* acc, const float* x, int64_t n, void* stream);
 
 /* y (bf16, n) = x (fp32, n) rounded to nearest even; n a multiple of 8, both 16-byte aligned. */
 int fa_convert_f32_bf16(const float* x, void* y, int64_t n, void* stream);

@@ -187,3 +187,40 @@ def test_variant_and_probe_host_validation(lib):
     assert lib.fa_set_backward_variant(-1) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_sm_clock_probe(None, None) == _lib.FA_ERR_INVALID_ARG
     assert lib.fa_sm_clock_probe(ctypes.c_void_p(0x100004), None) == _lib.FA_ERR_ALIGNMENT
+
+
+def test_accumulating_forward_and_backward_pieces_host_validation(lib):
+    A = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(8)]
+    ws = lib.fa_bwd_qk_workspace_size(1, 2, 256, 64)
+
+    def facc(q=A[0], k=A[1], v=A[2], o=A[3], l=A[4], first=1, d=64, causal=0, Hkv=2):
+        return lib.fa_fwd_accumulate(q, k, v, o, l, 1, 2, Hkv, 256, 256, d, 0.125, causal, first, None)
+
+    assert facc(first=2) == _lib.FA_ERR_INVALID_ARG
+    assert facc(o=None) == _lib.FA_ERR_INVALID_ARG
+    assert facc(l=MIS) == _lib.FA_ERR_ALIGNMENT
+    assert facc(d=96) == _lib.FA_ERR_UNSUPPORTED
+    assert facc(Hkv=3) == _lib.FA_ERR_INVALID_ARG                  # Hq not a multiple of Hkv
+    assert facc(o=ctypes.c_void_p(0x100000)) == _lib.FA_ERR_INVALID_ARG   # O_acc aliases Q
+
+    def prep(o=A[0], do=A[1], l=A[2], w=A[3], wsb=ws):
+        return lib.fa_bwd_prepare(o, do, l, w, wsb, 1, 2, 256, 64, None)
+
+    assert prep(w=None) == _lib.FA_ERR_INVALID_ARG
+    assert prep(wsb=ws - 1) == _lib.FA_ERR_INVALID_ARG
+    assert prep(do=MIS) == _lib.FA_ERR_ALIGNMENT
+    assert prep(w=ctypes.c_void_p(0x100000)) == _lib.FA_ERR_INVALID_ARG  # workspace aliases O
+
+    def acc(q=A[0], k=A[1], v=A[2], do=A[3], w=A[4], dk=A[5], dv=A[6], first=0, wsb=ws):
+        return lib.fa_bwd_accumulate(q, k, v, do, w, wsb, dk, dv, 1, 2, 2, 256, 256, 64, 0.125, 1, first, None)
+
+    assert acc(first=-1) == _lib.FA_ERR_INVALID_ARG
+    assert acc(dk=None) == _lib.FA_ERR_INVALID_ARG
+    assert acc(dv=MIS) == _lib.FA_ERR_ALIGNMENT
+    assert acc(wsb=16) == _lib.FA_ERR_INVALID_ARG
+    assert acc(dk=ctypes.c_void_p(0x700000)) == _lib.FA_ERR_INVALID_ARG  # dK_acc aliases dV_acc
+
+    assert lib.fa_bwd_finish(None, ws, A[0], 1, 2, 256, 64, 0.125, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_finish(A[1], ws - 16, A[0], 1, 2, 256, 64, 0.125, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_finish(A[1], ws, A[1], 1, 2, 256, 64, 0.125, None) == _lib.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_finish(A[1], ws, A[0], 0, 2, 256, 64, 0.125, None) == _lib.FA_OK  # empty

@@ -1,5 +1,6 @@
-"""GPU parity of the ring (context-parallel) pieces: the log-sum-exp merge, the fp32 helpers,
-and the whole ring forward / backward for R ranks emulated in one process on one GPU (the
+"""GPU parity of the ring (context-parallel) pieces: the log-sum-exp merge, the accumulating
+forward and backward entry points over several key blocks, the fp32 helpers, and the whole
+ring forward / backward (zig-zag layout) for R ranks emulated in one process on one GPU (the
 same per-rank steps as the distributed driver; the chunks are handed over in Python)."""
 import math
 
@@ -81,18 +82,69 @@ def test_accumulate_and_convert():
     assert torch.equal(out, acc.to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("world,causal", [(2, True), (4, True), (4, False)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_accumulating_calls_over_key_blocks_equal_full_attention(d, causal):
+    # fa_fwd_accumulate / fa_bwd_accumulate over three key blocks (the causal square last, so the
+    # earlier blocks are entirely visible) against the oracle on the whole key set
+    B, H, Nq = 1, 3, 384
+    blocks = [256, 384, 384]  # the last block holds the queries' own keys
+    Nk = sum(blocks)
+    dev, f64 = _seq(34, B, H, Nk, d)
+    q, do = dev["q"][:, :, Nk - Nq:].contiguous(), dev["do"][:, :, Nk - Nq:].contiguous()
+    scale = 1.0 / math.sqrt(d)
+    o_acc = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    l_acc = torch.full(q.shape[:-1], float("nan"), dtype=torch.float32, device="cuda")
+    starts = np.cumsum([0] + blocks[:-1])
+    kb = [(dev["k"][:, :, s:s + n].contiguous(), dev["v"][:, :, s:s + n].contiguous()) for s, n in zip(starts, blocks)]
+    for i, (k, v) in enumerate(kb):
+        last = i == len(kb) - 1
+        api.fa_fwd_accumulate(q, k, v, o_acc, l_acc, scale, causal and last, first=(i == 0))
+    o = api.fa_convert_f32_bf16(o_acc)
+    ws = api.fa_bwd_prepare(o, do, l_acc)
+    dk_acc = [torch.full(k.shape, float("nan"), dtype=torch.float32, device="cuda") for k, _ in kb]
+    dv_acc = [torch.full(k.shape, float("nan"), dtype=torch.float32, device="cuda") for k, _ in kb]
+    for i, (k, v) in enumerate(kb):
+        last = i == len(kb) - 1
+        api.fa_bwd_accumulate(q, k, v, do, ws, dk_acc[i], dv_acc[i], scale, causal and last, first=True)
+        api.fa_bwd_accumulate(q, k, v, do, ws, dk_acc[i], dv_acc[i], scale, causal and last, first=False)
+    dq = api.fa_bwd_finish(ws, B, H, Nq, d, scale)
+    # every block ran twice in the backward: dQ, dK and dV are twice the gradients
+    O, L = o_acc.double().cpu().numpy(), l_acc.double().cpu().numpy()
+    dQ = bf16_to_f64(dq) / 2.0
+    dK = np.concatenate([a.double().cpu().numpy() for a in dk_acc], axis=2) / 2.0
+    dV = np.concatenate([a.double().cpu().numpy() for a in dv_acc], axis=2) / 2.0
+    for h in range(H):
+        x = {k: f64[k][0, h] for k in f64}
+        o_ref, l_ref = OR.fwd(x["q"][Nk - Nq:], x["k"], x["v"], scale, causal)
+        dq_ref, dk_ref, dv_ref, _, _ = OR.bwd(x["q"][Nk - Nq:], x["k"], x["v"], x["do"][Nk - Nq:], scale, causal)
+        assert np.abs(O[0, h] - o_ref).max() <= TOL_O
+        assert np.abs(L[0, h] - l_ref).max() <= TOL_LSE
+        assert rel_l2(dQ[0, h], dq_ref) <= TOL_GRAD
+        assert rel_l2(dK[0, h], dk_ref) <= TOL_GRAD
+        assert rel_l2(dV[0, h], dv_ref) <= TOL_GRAD
+
+
+def test_accumulate_f32():
+    x = torch.randn(4096, device="cuda")
+    acc = torch.randn(4096, device="cuda")
+    want = acc + x
+    api.fa_accumulate_f32(acc, x)
+    assert torch.equal(acc, want)
+
+
+@pytest.mark.parametrize("world,causal", [(2, True), (4, True), (4, False), (3, True)])
 def test_emulated_ring_matches_oracle(world, causal):
     B, H, n, d = 1, 4, 512, 128
     N = n * world
     dev, f64 = _seq(33, B, H, N, d)
     scale = 1.0 / math.sqrt(d)
-    ch = {k: [t[:, :, r * n:(r + 1) * n].contiguous() for r in range(world)] for k, t in dev.items()}
+    ch = {k: [ring.zigzag_shard(t, r, world) for r in range(world)] for k, t in dev.items()}
     os_, lses = ring.ring_attention_fwd_emulated(ch["q"], ch["k"], ch["v"], scale, causal)
     dqs, dks, dvs = ring.ring_attention_bwd_emulated(ch["q"], ch["k"], ch["v"], os_, ch["do"], lses, scale, causal)
-    O = np.concatenate([bf16_to_f64(o) for o in os_], axis=2)
-    L = np.concatenate([l.double().cpu().numpy() for l in lses], axis=2)
-    dQ, dK, dV = (np.concatenate([bf16_to_f64(t) for t in ts], axis=2) for ts in (dqs, dks, dvs))
+    O = bf16_to_f64(ring.zigzag_unshard(os_))
+    L = ring.zigzag_unshard(lses).double().cpu().numpy()
+    dQ, dK, dV = (bf16_to_f64(ring.zigzag_unshard(ts)) for ts in (dqs, dks, dvs))
     worst = dict(O=0.0, LSE=0.0, dQ=0.0, dK=0.0, dV=0.0)
     for h in range(H):
         qr, kr = sample_rows(N, 96, h), sample_rows(N, 96, h + 50)
