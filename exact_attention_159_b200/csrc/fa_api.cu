@@ -271,7 +271,7 @@ int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   auto kern = gen ? fa::bwd_kernel<D, C, kBwdPoly16, true> : fa::bwd_kernel<D, C, kBwdPoly16, false>;
   if (set_smem(kern, L::kBytes) != cudaSuccess) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(prm.BHkv) * static_cast<unsigned>(prm.n_kv_tiles);
-  kern<<<grid, 384, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);
+  kern<<<grid, L::kThreads, L::kBytes, st>>>(q, k, v, dO, dq_acc, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

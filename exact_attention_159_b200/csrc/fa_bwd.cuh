@@ -74,11 +74,15 @@ struct BwdLayout {
   static constexpr bool kAliasDQ = (D == 128);
   static constexpr uint32_t kColDK = 0, kColDV = D, kColS = 2 * D, kColDP = 2 * D + 128;
   static constexpr uint32_t kColDQ = kAliasDQ ? kColDP : 2 * D + 256;
+  static constexpr int kThreads = 384;  // 12 warps: control, P/dS, dQ drain
 };
 
 // Register split (setmaxnreg): 128 * (80 + 240 + 184) = 384 * 168, the launch's total.  Each
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
 constexpr int kBwdRegsCtl = 80, kBwdRegsP = 240, kBwdRegsDQ = 184;
+constexpr int kBwdLaunchRegs = (65536 / 384) / 8 * 8;  // per-thread registers at launch (384 threads)
+static_assert(128 * (kBwdRegsCtl + kBwdRegsP + kBwdRegsDQ) <= 384 * kBwdLaunchRegs,
+              "backward register split exceeds the launch's registers");
 
 // GEN: grouped-query heads and / or Nq != Nk; without it (one query head per key/value head,
 // Nq == Nk) the group and offset terms are compile-time constants.
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(384, 1)
   const Guard g{abort_flag, prm.status};
 
   if (warp < 4) {
-    regs_dec<kBwdRegsCtl>();
+    regs_to<kBwdRegsCtl, kBwdLaunchRegs>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp < 8) {
-    regs_inc<kBwdRegsP>();
+    regs_to<kBwdRegsP, kBwdLaunchRegs>();
     // --------------------------------------------------- P^T and dS^T rows
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // key row within the tile
@@ -444,7 +448,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else {
-    regs_inc<kBwdRegsDQ>();
+    regs_to<kBwdRegsDQ, kBwdLaunchRegs>();
     // ---------------------------------------------------------- dQ drain
     // dQ_m (fp32, in TMEM) leaves 32 columns at a time through a swizzled shared-memory staging
     // buffer and a TMA reduce-add into the fp32 accumulator (two buffers, ping-pong).

@@ -154,7 +154,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const Guard g{abort_flag, prm.status};
 
   if (warp < 4) {
-    regs_dec<kBwdRegsCtl>();
+    regs_to<kBwdRegsCtl, kBwdLaunchRegs>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer (both CTAs)
       if (lane == 0) {
@@ -294,7 +294,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       }
     }
   } else if (warp < 8) {
-    regs_inc<kBwdRegsP>();
+    regs_to<kBwdRegsP, kBwdLaunchRegs>();
     // --------------------------------------------------- P^T and dS^T rows (both CTAs)
     const int quarter = warp & 3;
     const int j = quarter * 32 + lane;  // key row within this CTA's tile
@@ -440,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       }
     }
   } else {
-    regs_inc<kBwdRegsDQ>();
+    regs_to<kBwdRegsDQ, kBwdLaunchRegs>();
     // ---------------------------------------------------------- dQ drain (both CTAs)
     // This CTA's 64 query rows of dQ_m: lane l < 64 holds row l, columns 0..63 of d; lane l >= 64
     // row l - 64, columns 64..127.  They leave 32 columns at a time through two 8 KB staging

@@ -78,6 +78,7 @@ struct FwdLayout {
   static constexpr int kXchg = kMisc + 16;     // [tile][half][row] fp32 row-max / row-sum exchange
   static constexpr int kBytes = kXchg + 2 * 2 * 128 * 4;  // the dynamic shared memory base is 1024-byte aligned
   static constexpr int kThreads = 640;
+  static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;  // per-thread registers at launch
 };
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight async work).
@@ -91,6 +92,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // Register split (setmaxnreg): 128 * 56 + 512 * 104 <= 640 * 96, the launch's total.  Each
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
 constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 104;
+static_assert(128 * kFwdRegsCtl + 512 * kFwdRegsSoftmax <= 640 * 96, "forward register split exceeds the launch's");
 
 // GEN: grouped-query heads and / or N != Nk; without it (one query head per key/value head,
 // N == Nk) the group and offset terms are compile-time constants.
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(640, 1)
   const uint32_t tmem = *tmem_slot;
   const Guard g{abort_flag, prm.status};
   if (warp < 4) {
-    regs_dec<kFwdRegsCtl>();
+    regs_to<kFwdRegsCtl, L::kLaunchRegs>();
     if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nkv_max > 0) {
@@ -259,7 +261,7 @@ __global__ void __launch_bounds__(640, 1)
     }
     }
   } else {
-    regs_inc<kFwdRegsSoftmax>();
+    regs_to<kFwdRegsSoftmax, L::kLaunchRegs>();
     // ------------------------------------------- softmax / correction / epilogue
     const int t = (warp - 4) >> 3;        // query tile
     const int h = ((warp - 4) >> 2) & 1;  // which 64 key columns of the row (and D/2 columns of O)

@@ -123,7 +123,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
   const Guard g{abort_flag, prm.status};
 
   if (warp < 4) {
-    regs_dec<kFwdRegsCtl>();
+    regs_to<kFwdRegsCtl, (65536 / L::kThreads) / 8 * 8>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
@@ -208,7 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
       }
     }
   } else {
-    regs_inc<kFwdRegsSoftmax>();
+    regs_to<kFwdRegsSoftmax, (65536 / L::kThreads) / 8 * 8>();
     // ------------------------------------------- softmax / correction / epilogue
     const int t = (warp - 4) >> 3;
     const int h = ((warp - 4) >> 2) & 1;

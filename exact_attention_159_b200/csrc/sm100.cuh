@@ -270,6 +270,14 @@ template <int N>
 __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Moves a warpgroup from the launch's per-thread register count LAUNCH to N: .dec when N is below
+// it, .inc when above (setmaxnreg.inc may only raise the count and .dec only lower it).
+template <int N, int LAUNCH>
+__device__ __forceinline__ void regs_to() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count out of range");
+  if constexpr (N < LAUNCH) regs_dec<N>();
+  else if constexpr (N > LAUNCH) regs_inc<N>();
+}
 
 // max(a, b, c) in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
