@@ -23,7 +23,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 // Forward: element pairs out of every 16 whose exponentials take the FMA-pipe cubic by default,
 // per head dimension (index 0: d = 64, 1: d = 128).
-constexpr int kPolyDefault[2] = {0, 0};
+constexpr int kPolyDefault[2] = {4, 1};
 constexpr int kBwdPoly16 = 0;  // backward: the SFU alone measured faster than any polynomial share
 
 __device__ int g_status;  // first device-side failure (wait site), 0 = none

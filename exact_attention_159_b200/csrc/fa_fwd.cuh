@@ -8,16 +8,15 @@
 //   warp 0        TMA producer: Q tiles once, then a ring of K/V tiles
 //   warp 1        MMA issuer (one thread) and TMEM owner
 //   warps 2, 3    idle (they complete the first warpgroup)
-//   warps 4..11   softmax + correction + epilogue for query tile 0
-//   warps 12..19  the same for query tile 1
-// Every score row is split between two threads (two warps on the same TMEM
-// lane quarter): each takes 64 of the 128 key columns, and the pair agrees on
-// the row maximum through shared memory and a 64-thread hardware barrier that
-// also ANDs the pair's "every wait succeeded" flags (bar.red.and), so a failed
-// wait makes both warps leave together.  Four
-// softmax warps per SM sub-partition hide the SFU and TMEM latencies.
-// Registers are re-split per warpgroup with setmaxnreg (56 / 104 of the
-// 96 x 640 launched).  The softmax arithmetic uses packed fp32x2 FMA/add.
+//   warps 4..7    softmax + correction + epilogue for query tile 0
+//   warps 8..11   the same for query tile 1
+// One thread owns one score row: it loads all 128 scores of its row for a key
+// tile into registers, so the row maximum and the row sum need no exchange
+// between threads, and its 128 independent exponentials give the instruction-
+// level parallelism that lets a share of them run as the cubic on the FMA
+// pipe alongside the SFU.  Registers are re-split per warpgroup with
+// setmaxnreg (56 for the control warps, 224 for the softmax warps, of the
+// 168 x 384 launched).  The softmax arithmetic uses packed fp32x2 FMA/add.
 // Tensor memory (512 columns x 128 lanes x 32 bit, "TMEM (256 KB per SM)"):
 //   S_t = Q_t K^T  fp32, 128 columns at 128*t; P_t (bf16, packed two per
 //   column) is written back over the first 64 columns of S_t and read from
@@ -75,9 +74,8 @@ struct FwdLayout {
   // q, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain
   static constexpr int kNumBars = 1 + 4 * kStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kXchg = kMisc + 16;     // [tile][half][row] fp32 row-max / row-sum exchange
-  static constexpr int kBytes = kXchg + 2 * 2 * 128 * 4;  // the dynamic shared memory base is 1024-byte aligned
-  static constexpr int kThreads = 640;
+  static constexpr int kBytes = kMisc + 16;  // the dynamic shared memory base is 1024-byte aligned
+  static constexpr int kThreads = 384;
   static constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;  // per-thread registers at launch
 };
 
@@ -89,15 +87,16 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Register split (setmaxnreg): 128 * 56 + 512 * 104 <= 640 * 96, the launch's total.  Each
+// Register split (setmaxnreg): 128 * 56 + 256 * 224 = 384 * 168, the launch's total.  Each
 // setmaxnreg heads its role's branch so the register budget of that code is unambiguous.
-constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 104;
-static_assert(128 * kFwdRegsCtl + 512 * kFwdRegsSoftmax <= 640 * 96, "forward register split exceeds the launch's");
+constexpr int kFwdRegsCtl = 56, kFwdRegsSoftmax = 224;
+static_assert(128 * kFwdRegsCtl + 256 * kFwdRegsSoftmax <= 384 * ((65536 / 384) / 8 * 8),
+              "forward register split exceeds the launch's");
 
 // GEN: grouped-query heads and / or N != Nk; without it (one query head per key/value head,
 // N == Nk) the group and offset terms are compile-time constants.
 template <int D, bool CAUSAL, int POLY16, bool GEN>
-__global__ void __launch_bounds__(640, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams prm) {
   using L = FwdLayout<D>;
@@ -152,7 +151,7 @@ __global__ void __launch_bounds__(640, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 256);
+      mbar_init(&p_full[t], 128);
       mbar_init(&o_full[t], 1);
     }
     mbar_init(drain, 1);
@@ -263,75 +262,69 @@ __global__ void __launch_bounds__(640, 1)
   } else {
     regs_to<kFwdRegsSoftmax, L::kLaunchRegs>();
     // ------------------------------------------- softmax / correction / epilogue
-    const int t = (warp - 4) >> 3;        // query tile
-    const int h = ((warp - 4) >> 2) & 1;  // which 64 key columns of the row (and D/2 columns of O)
-    const int quarter = warp & 3;         // TMEM lanes this warp may touch: 32*quarter .. +31
+    // One thread per score row: warps 4..7 hold the 128 rows of query tile 0 (one TMEM lane
+    // quarter each), warps 8..11 those of tile 1.  A thread keeps its whole row of 128 scores in
+    // registers, so the row maximum needs no exchange with another thread.
+    const int t = (warp - 4) >> 2;   // query tile
+    const int quarter = warp & 3;    // TMEM lanes this warp may touch: 32*quarter .. +31
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + 128 * t + lane_off;
-    const uint32_t tO = tmem + 256 + D * t + (D / 2) * h + lane_off;
-    float* xchg = reinterpret_cast<float*>(smem + L::kXchg) + t * 256;  // [half][row]
-    const int bar_id = 1 + 4 * t + quarter;                            // the two warps sharing these rows
+    const uint32_t tO = tmem + 256 + D * t + lane_off;
     const int qt = 2 * pair + t;
     const int row = qt * kTile + r;  // query row within the head
     const float sl2 = prm.scale_log2;
-    float m_ref = -INFINITY, l = 0.0f;  // l: this thread's half of the row sum
+    float m_ref = -INFINITY, l = 0.0f;
     bool ok = true;
     for (int j = 0; j < nkv[t]; ++j) {
-      // every exit decision is taken jointly by the two warps of a row (group_and), so neither is
-      // ever left waiting at a barrier the other skipped; after a failed wait the block below
-      // only reads stale TMEM columns of this CTA's own allocation before the joint exit
-      const bool okl = ok && wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7);
+      if (!(ok = wait_warp(&s_full[t], j & 1, g, kSiteFwd | 7))) break;
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tS + 64 * h, sr[0]);
-      tmem_ld32(tS + 64 * h + 32, sr[1]);
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sr[c]);
       tmem_wait_ld();
-      reg_fence(sr[0]);
-      reg_fence(sr[1]);
-      // scores stay in the registers tcgen05.ld wrote (S(c) reads local column c as fp32)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+      // scores stay in the registers tcgen05.ld wrote (S(c) reads key column c as fp32)
 #define S(c) __uint_as_float(sr[(c) >> 5][(c) & 31])
       // masking: keys past the end, and (causal) keys beyond the first row's reach
       const bool edge = (CAUSAL && j * kTile + kTile - 1 > qt * kTile + off) || ((j + 1) * kTile > Nk);
       if (edge) {
-        const int key0 = j * kTile + 64 * h;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = key0 + c;
+        for (int c = 0; c < kTile; ++c) {
+          const int key = j * kTile + c;
           if (key >= Nk || (CAUSAL && key > row + off)) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
         }
       }
-      // row maximum: two chains of 3-input max over this half, then the partner's half
-      float mx[2] = {S(0), S(32)};
+      // row maximum: four chains of 3-input max
+      float mx[4];
 #pragma unroll
-      for (int q = 0; q < 2; ++q)
+      for (int q = 0; q < 4; ++q) {
+        mx[q] = S(32 * q);
 #pragma unroll
         for (int c = 32 * q + 1; c < 32 * q + 31; c += 2) mx[q] = fmax3(mx[q], S(c), S(c + 1));
-#pragma unroll
-      for (int q = 0; q < 2; ++q) mx[q] = fmaxf(mx[q], S(32 * q + 31));
-      const float mine = fmaxf(mx[0], mx[1]);
-      xchg[128 * h + r] = mine;
-      if (!(ok = group_and(bar_id, 64, okl))) break;
-      const float m_new = fmaxf(m_ref, fmaxf(mine, xchg[128 * (h ^ 1) + r]) * sl2);
-      const bool need = m_new > m_ref + prm.tau;  // identical in both threads of the row
+        mx[q] = fmaxf(mx[q], S(32 * q + 31));
+      }
+      const float m_new = fmaxf(m_ref, fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2);
+      const bool need = m_new > m_ref + prm.tau;
       const float alpha = need ? exp2_sfu(m_ref - m_new) : 1.0f;
       if (need) {
         l *= alpha;
         m_ref = m_new;
       }
-      // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 columns at a time)
+      // P = 2^(S * scale * log2e - m_ref), row sum, bf16 P back over S (32 keys -> 16 columns at a time)
       // a row that has seen no key yet (m_ref = -inf; causal with N > Nk) has only masked scores
       const float m_sub = GEN && m_ref == -INFINITY ? 0.0f : m_ref;
       const float2 c2 = make_float2(sl2, sl2), nm2 = make_float2(-m_sub, -m_sub);
       float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
-      // The two paths are separate code, so the tiles that use the cubic for part of their
-      // exponentials issue no SFU operation for that part (a select between the two would).
       // POLY16 of every 16 element pairs (evenly spaced) take the cubic
       constexpr int kPolyStride = POLY16 > 0 ? 16 / POLY16 : 16;
+      // The two paths are separate code, so the tiles that use the cubic for part of their
+      // exponentials issue no SFU operation for that part (a select between the two would).
       auto exp_store = [&](auto poly_tag) {
         constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -350,7 +343,7 @@ __global__ void __launch_bounds__(640, 1)
               ls0 = __fadd2_rn(ls0, p);
             pk[e] = pack_bf16x2(p.x, p.y);
           }
-          tmem_st16(tS + 32 * h + 16 * cc, pk);
+          tmem_st16(tS + 16 * cc, pk);
         }
       };
       if (POLY16 > 0 && !edge)  // masked (edge) tiles keep exact zeros from the SFU
@@ -361,56 +354,50 @@ __global__ void __launch_bounds__(640, 1)
       const float2 ls = __fadd2_rn(ls0, ls1);
       l += ls.x + ls.y;
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // correction: this thread's half of O_t *= alpha once the previous P.V has landed (before
+        // correction: this thread's row of O_t *= alpha once the previous P.V has landed (before
         // p_full lets the next P.V accumulate into it)
         ok = wait_warp(&o_full[t], (j - 1) & 1, g, kSiteFwd | 8);
-        tc_fence_after();  // a failed wait is carried to the next joint decision
+        tc_fence_after();
+        if (ok) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
-          reg_fence(o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+            reg_fence(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      if (ok) mbar_arrive(&p_full[t]);
+      if (!ok) break;
+      mbar_arrive(&p_full[t]);
     }
-    float lse_old = -INFINITY;  // accumulating calls: the row's LSE over the key blocks folded so far
-    if (nkv[t] > 0) {
-      // full row sum from the two halves (joint decision, as in the loop)
-      const bool okl = ok && wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
-      if (okl) {
-        tc_fence_after();
-        xchg[128 * h + r] = l;
-      }
-      // both threads of the row read the old LSE before the barrier; it is replaced after it
-      if (prm.O_acc != nullptr && !prm.acc_first && row < prm.N)
-        lse_old = prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row];
-      ok = group_and(bar_id, 64, okl);
-    }
+    if (ok && nkv[t] > 0) ok = wait_warp(&o_full[t], (nkv[t] - 1) & 1, g, kSiteFwd | 9);
     if (ok && nkv[t] > 0 && prm.O_acc != nullptr) {
       // fold into the fp32 accumulators: L = ln(e^LSE_old + e^LSE), O_acc = e^(LSE_old - L) O_acc +
-      // e^(LSE - L) O (a side at -inf weighs 0; both at -inf leave O_acc = 0, LSE_acc = -inf)
-      const float l_row = l + xchg[128 * (h ^ 1) + r];
-      const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+      // e^(LSE - L) O (a side at -inf weighs 0; both at -inf leave O_acc = 0, LSE_acc = -inf); the
+      // row's thread alone reads and replaces its LSE
+      tc_fence_after();
+      const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
       const bool store = row < prm.N;
-      const float lse = l_row > 0.0f ? (m_ref + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+      const size_t ri = static_cast<size_t>(bh) * prm.N + (store ? row : 0);
+      const float lse = l > 0.0f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       float lse_new = lse, wa = 0.0f, wb = 1.0f;
-      if (!prm.acc_first) {
+      if (!prm.acc_first && store) {
+        const float lse_old = prm.LSE_acc[ri];
         const float mx = fmaxf(lse_old, lse);
         lse_new = mx == -INFINITY ? -INFINITY : mx + log1pf(expf(-fabsf(lse_old - lse)));
         wa = lse_new == -INFINITY ? 0.0f : expf(lse_old - lse_new);
         wb = lse_new == -INFINITY ? 0.0f : expf(lse - lse_new);
       }
       const float scale_b = inv_l * wb;
-      float* arow = prm.O_acc + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D + (D / 2) * h;
+      float* arow = prm.O_acc + ri * D;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_wait_ld();
@@ -432,14 +419,14 @@ __global__ void __launch_bounds__(640, 1)
           }
         }
       }
-      if (store && h == 0) prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row] = lse_new;
+      if (store) prm.LSE_acc[ri] = lse_new;
     } else if (ok && nkv[t] > 0) {
-      const float l_row = l + xchg[128 * (h ^ 1) + r];
-      const float inv_l = l_row > 0.0f ? 1.0f / l_row : 0.0f;  // a row that sees no key: O = 0, LSE = -inf
+      tc_fence_after();
+      const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;  // a row that sees no key: O = 0, LSE = -inf
       const bool store = row < prm.N;
-      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D + (D / 2) * h;
+      __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + (store ? row : 0)) * D;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * c, o);
         tmem_wait_ld();
@@ -454,26 +441,25 @@ __global__ void __launch_bounds__(640, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (store && h == 0)
+      if (store)
         prm.LSE[static_cast<size_t>(bh) * prm.N + row] =
-            l_row > 0.0f ? (m_ref + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+            l > 0.0f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     } else if (nkv[t] == 0 && qt < n_tiles && row < prm.N) {
       // a query tile no key is visible to (causal, N > Nk): O = 0, LSE = -inf (an accumulating call
       // that is not the first adds nothing)
       if (prm.O_acc == nullptr) {
-        __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
+        __nv_bfloat16* orow = prm.O + (static_cast<size_t>(bh) * prm.N + row) * D;
 #pragma unroll
-        for (int i = 0; i < D / 16; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (h == 0) prm.LSE[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
+        for (int i = 0; i < D / 8; ++i) reinterpret_cast<uint4*>(orow)[i] = make_uint4(0u, 0u, 0u, 0u);
+        prm.LSE[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
       } else if (prm.acc_first) {
-        float* arow = prm.O_acc + (static_cast<size_t>(bh) * prm.N + row) * D + (D / 2) * h;
+        float* arow = prm.O_acc + (static_cast<size_t>(bh) * prm.N + row) * D;
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) reinterpret_cast<float4*>(arow)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (h == 0) prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
+        for (int i = 0; i < D / 4; ++i) reinterpret_cast<float4*>(arow)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        prm.LSE_acc[static_cast<size_t>(bh) * prm.N + row] = -INFINITY;
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

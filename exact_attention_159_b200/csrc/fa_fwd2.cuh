@@ -54,6 +54,11 @@ struct Fwd2Params {
   int* status;
 };
 
+// Register split (setmaxnreg) of the pair kernel: 128 * 56 + 512 * 104 <= 640 * 96, the launch's total.
+constexpr int kFwd2RegsCtl = 56, kFwd2RegsSoftmax = 104;
+static_assert(128 * kFwd2RegsCtl + 512 * kFwd2RegsSoftmax <= 640 * ((65536 / 640) / 8 * 8),
+              "pair forward register split exceeds the launch's");
+
 template <bool CAUSAL, int POLY16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
     fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK64,
@@ -123,7 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
   const Guard g{abort_flag, prm.status};
 
   if (warp < 4) {
-    regs_to<kFwdRegsCtl, (65536 / L::kThreads) / 8 * 8>();
+    regs_to<kFwd2RegsCtl, (65536 / L::kThreads) / 8 * 8>();
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
@@ -208,7 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
       }
     }
   } else {
-    regs_to<kFwdRegsSoftmax, (65536 / L::kThreads) / 8 * 8>();
+    regs_to<kFwd2RegsSoftmax, (65536 / L::kThreads) / 8 * 8>();
     // ------------------------------------------- softmax / correction / epilogue
     const int t = (warp - 4) >> 3;
     const int h = ((warp - 4) >> 2) & 1;
