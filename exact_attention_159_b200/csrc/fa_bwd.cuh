@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(384, 1)
   const int off = GEN ? prm.off : 0;
   const int Nk = GEN ? prm.Nk : prm.N;
   int bkv, n;  // key tile n = 0 (the most causal work) first, a few heads at a time
-  cta_order(blockIdx.x, prm.BHkv, prm.n_kv_tiles, bkv, n);
+  cta_order(blockIdx.x, prm.BHkv, prm.n_kv_tiles, cta_head_group(prm.BHkv, prm.n_kv_tiles, CAUSAL), bkv, n);
   // first query tile that sees key tile n: its last row + off reaches the tile's first key
   int m_begin = 0;
   if (CAUSAL) {

@@ -113,7 +113,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_units = (prm.n_kv_tiles + 1) / 2;
   int bh, u;  // key-tile pair u = 0 (the most causal work) first, a few heads at a time
-  cta_order(blockIdx.x >> 1, prm.BHkv, n_units, bh, u);
+  cta_order(blockIdx.x >> 1, prm.BHkv, n_units, cta_head_group(prm.BHkv, n_units, CAUSAL), bh, u);
   const int n0 = 2 * u, n = n0 + r;                  // this CTA's key tile (n1 may lie past the end)
   const int m_begin = CAUSAL ? n0 : 0;               // first query tile that sees key tile n0
   const int n_it = prm.n_q_tiles - m_begin;          // >= 1

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int bh, unit;  // heaviest causal work (the last query tiles) first, a few heads at a time
-  cta_order(blockIdx.x, prm.BH, prm.n_pairs, bh, unit);
+  cta_order(blockIdx.x, prm.BH, prm.n_pairs, cta_head_group(prm.BH, prm.n_pairs, CAUSAL), bh, unit);
   const int pair = prm.n_pairs - 1 - unit;
   const int Nk = GEN ? prm.Nk : prm.N;
   const int off = GEN ? prm.off : 0;

@@ -89,7 +89,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(640, 1)
   const uint32_t rank = cluster_rank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int bh, unit;
-  cta_order(blockIdx.x >> 1, prm.BH, prm.n_quads, bh, unit);
+  cta_order(blockIdx.x >> 1, prm.BH, prm.n_quads, cta_head_group(prm.BH, prm.n_quads, CAUSAL), bh, unit);
   const int quad = prm.n_quads - 1 - unit;  // heaviest causal work first
   const int n_tiles = (prm.N + kTile - 1) / kTile;
   int nkv[2];

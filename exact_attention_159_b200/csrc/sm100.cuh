@@ -286,16 +286,32 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// CTA order for causal work lists: heads are taken in groups of kHeadGroup (so the CTAs running
-// at one time share a few heads' streamed tiles in L2), heaviest unit first inside a group with the
-// head as the fast index.  Returns the head and the unit index (0 = heaviest).
+// CTA order for causal work lists: heads are taken in groups (so the CTAs running at one time share
+// a few heads' streamed tiles in L2), heaviest unit first inside a group with the head as the fast
+// index.  Returns the head and the unit index (0 = heaviest).
 constexpr int kHeadGroup = 2;
-__device__ __forceinline__ void cta_order(int cta, int n_heads, int n_units, int& head, int& unit) {
-  const int g = cta / (kHeadGroup * n_units);
-  const int heads_here = min(kHeadGroup, n_heads - g * kHeadGroup);
-  const int r = cta - g * kHeadGroup * n_units;
+__device__ __forceinline__ void cta_order(int cta, int n_heads, int n_units, int group, int& head, int& unit) {
+  const int g = cta / (group * n_units);
+  const int heads_here = min(group, n_heads - g * group);
+  const int r = cta - g * group * n_units;
   unit = r / heads_here;
-  head = g * kHeadGroup + r % heads_here;
+  head = g * group + r % heads_here;
+}
+// Heads per group.  Two keep the resident CTAs on few heads' tiles.  With causal work a head's units
+// range from 1 to n_units steps and its heaviest unit is about 2 / (n_units + 1) of the head's work;
+// it is scheduled first in its group, and it must not outlast the rest of the group's work spread
+// over the other SMs, or the last group's heavy units run on alone at the end of the launch.  A
+// group of g heads holds g / (2 / (n_units + 1)) heaviest units of work, so g = 256 / (n_units + 1)
+// (rounded up, at least two) covers about 128 SMs; g is then lowered to a divisor of the head
+// count, since a short last group would end the launch on its own.  Long sequences keep two heads;
+// short ones take more heads per group (16 heads at 16384 rows: 4; 64 heads at 2048 rows: 16).
+__device__ __forceinline__ int cta_head_group(int n_heads, int n_units, bool causal) {
+  if (!causal) return kHeadGroup;
+  int g = (256 + n_units) / (n_units + 1);
+  g = g < kHeadGroup ? kHeadGroup : g;
+  g = g > n_heads ? n_heads : g;
+  while (g > 1 && n_heads % g != 0) --g;
+  return g;
 }
 
 // ------------------------------------------------------- cluster pair (2 SMs)
