@@ -29,15 +29,20 @@ def bf16_to_f64(t) -> np.ndarray:
 
 
 def sample_rows(N: int, count: int, seed: int) -> np.ndarray:
-    """Tile edges, both ends, and seeded random rows."""
-    fixed = [0, 1, 2, N - 1, N - 2]
-    for t in range(128, N, 128):
-        if len(fixed) > count // 2:
-            break
-        fixed += [t - 1, t]
-    fixed = [x for x in fixed if 0 <= x < N]
-    rnd = np.random.default_rng(seed).choice(N, size=min(N, count), replace=False)
-    return np.unique(np.concatenate([np.array(fixed, dtype=np.int64), rnd.astype(np.int64)]))[:max(count, 1)]
+    """Rows to compare: both ends, the rows on either side of tile boundaries spread evenly over the
+    whole length, then seeded random rows up to `count` in all (the fixed rows are always kept)."""
+    fixed = {0, 1, 2, N - 1, N - 2}
+    bounds = list(range(128, N, 128))
+    pairs = max(count // 2 - len(fixed), 0) // 2
+    if bounds and pairs:
+        step = -(-len(bounds) // pairs)
+        for t in bounds[::step]:
+            fixed.update((t - 1, t))
+    fixed = np.array(sorted(x for x in fixed if 0 <= x < N), dtype=np.int64)
+    rest = np.setdiff1d(np.arange(N, dtype=np.int64), fixed)
+    n_rnd = max(0, min(count - len(fixed), len(rest)))
+    rnd = np.random.default_rng(seed).choice(rest, size=n_rnd, replace=False) if n_rnd else rest[:0]
+    return np.unique(np.concatenate([fixed, rnd.astype(np.int64)]))
 
 
 def rel_l2(a, b) -> float:

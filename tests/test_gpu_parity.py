@@ -110,6 +110,20 @@ def test_long_context_forward_backward_32768():
         assert np.linalg.norm(dK[0, h].sum(0)) <= 0.05 * spread, f"head {h}: sum dK != 0"
 
 
+def test_causal_cta_groups_head_count_not_a_power_of_two():
+    """30 heads of 4096 causal rows: the causal CTA order takes the heads in groups sized to the
+    work per head and lowered to a divisor of the head count (15 heads per forward group, 6 per
+    backward group here).  Every head and every query and key tile must still be computed once:
+    each checked head has rows sampled in all of its query tiles and its first and last key tile
+    checked in full."""
+    c = Case(2, 15, 4096, 64, True, seed_workload=16, bwd=True)
+    o, lse = c.fwd_gpu()
+    heads = [(b, h) for b in range(2) for h in (0, 7, 14)]
+    check_fwd(c, o, lse, heads, 64, "fwd causal B2 H15 N4096 d64")
+    edge_keys = np.concatenate([np.arange(128), np.arange(c.N - 128, c.N)])
+    check_bwd(c, c.bwd_gpu(o, lse), heads, 64, 64, "bwd causal B2 H15 N4096 d64", extra_k=edge_keys)
+
+
 SWEEP = [(B, N, d, causal) for (B, N) in ((8, 2048), (2, 8192), (1, 16384)) for d in (64, 128)
          for causal in (False, True)]
 
