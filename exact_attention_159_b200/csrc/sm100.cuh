@@ -302,16 +302,22 @@ __device__ __forceinline__ void cta_order(int cta, int n_heads, int n_units, int
 // it is scheduled first in its group, and it must not outlast the rest of the group's work spread
 // over the other SMs, or the last group's heavy units run on alone at the end of the launch.  A
 // group of g heads holds g / (2 / (n_units + 1)) heaviest units of work, so g = 256 / (n_units + 1)
-// (rounded up, at least two) covers about 128 SMs; g is then lowered to a divisor of the head
-// count, since a short last group would end the launch on its own.  Long sequences keep two heads;
-// short ones take more heads per group (16 heads at 16384 rows: 4; 64 heads at 2048 rows: 16).
+// (rounded up, at least two) covers about 128 SMs.  g then becomes a divisor of the head count,
+// since a short last group would end the launch on its own: the largest divisor not above g, or,
+// when that is under g / 2, the smallest one above it.  Long sequences keep two heads; short ones
+// take more heads per group (16 heads at 16384 rows: 4; 64 heads at 2048 rows: 16; 11 heads at
+// 8192 rows: 11).
 __device__ __forceinline__ int cta_head_group(int n_heads, int n_units, bool causal) {
   if (!causal) return kHeadGroup;
   int g = (256 + n_units) / (n_units + 1);
   g = g < kHeadGroup ? kHeadGroup : g;
-  g = g > n_heads ? n_heads : g;
-  while (g > 1 && n_heads % g != 0) --g;
-  return g;
+  if (g >= n_heads) return n_heads;
+  int lo = g;
+  while (n_heads % lo != 0) --lo;
+  if (2 * lo >= g) return lo;
+  int hi = g + 1;
+  while (n_heads % hi != 0) ++hi;
+  return hi;
 }
 
 // ------------------------------------------------------- cluster pair (2 SMs)

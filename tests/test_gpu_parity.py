@@ -124,6 +124,17 @@ def test_causal_cta_groups_head_count_not_a_power_of_two():
     check_bwd(c, c.bwd_gpu(o, lse), heads, 64, 64, "bwd causal B2 H15 N4096 d64", extra_k=edge_keys)
 
 
+def test_causal_cta_groups_prime_head_count():
+    """11 heads of 8192 causal rows: no divisor of 11 lies near the group size the work per head
+    asks for (8 in the forward, 4 in the backward), so all 11 heads form one group."""
+    c = Case(1, 11, 8192, 64, True, seed_workload=17, bwd=True)
+    o, lse = c.fwd_gpu()
+    heads = [(0, 0), (0, 5), (0, 10)]
+    check_fwd(c, o, lse, heads, 64, "fwd causal B1 H11 N8192 d64")
+    edge_keys = np.concatenate([np.arange(128), np.arange(c.N - 128, c.N)])
+    check_bwd(c, c.bwd_gpu(o, lse), heads, 48, 48, "bwd causal B1 H11 N8192 d64", extra_k=edge_keys)
+
+
 SWEEP = [(B, N, d, causal) for (B, N) in ((8, 2048), (2, 8192), (1, 16384)) for d in (64, 128)
          for causal in (False, True)]
 
