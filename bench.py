@@ -270,7 +270,8 @@ def run_gpu(args):
     # The heads are independent, so the end-to-end step streams them in chunks: the copy of chunk
     # c+1's inputs and of chunk c-1's results overlap the kernels of chunk c (copy engines on their
     # own streams, ordered by events).  Every byte still crosses PCIe inside the timed region.
-    n_chunks = E2E_CHUNKS if (B == 1 and H % E2E_CHUNKS == 0) else 1
+    chunks = args.e2e_chunks
+    n_chunks = chunks if (B == 1 and chunks >= 1 and H % chunks == 0) else 1
     hc = H // n_chunks
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ws_c = torch.empty(api.fa_bwd_workspace_size(B, hc, N, d), dtype=torch.uint8, device="cuda")
@@ -652,6 +653,7 @@ def main():
     ap.add_argument("--shape", default="1,16,16384,128", help="B,H,N,d for --profile")
     ap.add_argument("--causal", type=int, default=1, help="causal flag for --profile")
     ap.add_argument("--source-hash", action="store_true", help="print the kernel source hash and exit")
+    ap.add_argument("--e2e-chunks", type=int, default=E2E_CHUNKS, help="head chunks of the end-to-end step")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.source_hash:
