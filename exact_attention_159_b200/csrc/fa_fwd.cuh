@@ -205,6 +205,11 @@ __global__ void __launch_bounds__(384, 1)
     }
     } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA
+    // One thread issues every UMMA, per key tile j in the order P.V(0, j), S(0, j+1), P.V(1, j),
+    // S(1, j+1): the order is what keeps the two tiles' softmax phases half a period apart.  The
+    // tensor pipe takes only about one instruction ahead of its issuing thread, so the barrier
+    // waits between batches cost pipe time (80-90 clocks per 64-clock UMMA here, with the softmax
+    // warps busy on the same SM); every way of sharing the issue between two threads was slower.
     if (lane == 0 && nkv_max > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // P (TMEM) x V (MN-major)
