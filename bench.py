@@ -468,7 +468,8 @@ def gpu_per_config(api, reps=5):
             row.update(bwd_ms=round(b_ms, 4), bwd_tflops=round(f_bwd / (b_ms * 1e-3) / 1e12, 2),
                        bwd_main_ms=round(m_ms, 4), bwd_main_tflops=round(f_bwd / (m_ms * 1e-3) / 1e12, 2))
         if wid == 4 and d == 128:
-            # the cluster-pair (cta_group::2) variants of both kernels on the same inputs, for comparison
+            # the cluster-pair (cta_group::2) variants of both kernels on the same inputs, for comparison;
+            # a failure here is reported in the row and leaves the other timings in place
             try:
                 api.fa_set_forward_variant(1)
                 fwd_call()
@@ -478,16 +479,18 @@ def gpu_per_config(api, reps=5):
                 if bwd:
                     bwd_call()
                 pb = [timed(bwd_call, 1) for _ in range(reps)] if bwd else []
+                torch.cuda.synchronize()
+                p_ms = statistics.median(e[0].elapsed_time(e[1]) for e in pe)
+                row.update(pair_fwd_ms=round(p_ms, 4), pair_fwd_tflops=round(f_fwd / (p_ms * 1e-3) / 1e12, 2))
+                if bwd:
+                    pm_ms = statistics.median(e[2].elapsed_time(e[3]) for e in pb)
+                    row.update(pair_bwd_main_ms=round(pm_ms, 4),
+                               pair_bwd_main_tflops=round(f_bwd / (pm_ms * 1e-3) / 1e12, 2))
+            except Exception as exc:  # noqa: BLE001 -- reported in the JSON line
+                row["pair_error"] = f"{type(exc).__name__}: {exc}"
             finally:
                 api.fa_set_forward_variant(0)
                 api.fa_set_backward_variant(0)
-            torch.cuda.synchronize()
-            p_ms = statistics.median(e[0].elapsed_time(e[1]) for e in pe)
-            row.update(pair_fwd_ms=round(p_ms, 4), pair_fwd_tflops=round(f_fwd / (p_ms * 1e-3) / 1e12, 2))
-            if bwd:
-                pm_ms = statistics.median(e[2].elapsed_time(e[3]) for e in pb)
-                row.update(pair_bwd_main_ms=round(pm_ms, 4),
-                           pair_bwd_main_tflops=round(f_bwd / (pm_ms * 1e-3) / 1e12, 2))
         rows.append(row)
         del x, o, lse, ws, grads
     return {"rows": rows, "inputs": "seeded N(0,1) bf16 drawn on the device (torch generator), stress "
